@@ -1,0 +1,154 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin fails.
+
+Each mutation replaces one oracle function with a wrong variant: a dropped
+term, a wrong sign, a transposed operand, a wrong normalisation, a reversed
+tie rule. The pins must reject every one of them.
+"""
+import numpy as np
+import pytest
+from scipy.special import erf
+
+import oracle.rs_oracle as rs_oracle
+from oracle_pins import ALL_PINS
+
+orig = {n: getattr(rs_oracle, n) for n in
+        ["layer_norm", "gelu", "fc", "mlp", "shift_score", "select_topk", "gather", "sublayer"]}
+
+
+def _ln_unbiased(x, gamma, beta, eps=rs_oracle.EPS):
+    mu = x.mean(axis=-1, keepdims=True)
+    var = x.var(axis=-1, ddof=1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * gamma + beta
+
+
+def _ln_no_beta(x, gamma, beta, eps=rs_oracle.EPS):
+    return orig["layer_norm"](x, gamma, np.zeros_like(beta), eps)
+
+
+def _ln_no_eps(x, gamma, beta, eps=rs_oracle.EPS):
+    return orig["layer_norm"](x, gamma, beta, 0.0)
+
+
+def _ln_no_gamma(x, gamma, beta, eps=rs_oracle.EPS):
+    return orig["layer_norm"](x, np.ones_like(gamma), beta, eps)
+
+
+def _gelu_no_sqrt2(z):
+    return 0.5 * z * (1.0 + erf(z))
+
+
+def _gelu_tanh(z):
+    return 0.5 * z * (1.0 + np.tanh(np.sqrt(2 / np.pi) * (z + 0.044715 * z ** 3)))
+
+
+def _fc_transposed(v, W, b):
+    return v @ W + b  # weight read as [in, out]: wrong for nn.Linear's [out, in]
+
+
+def _fc_no_bias(v, W, b):
+    return v @ W.T
+
+
+def _mlp_relu(u, W1, b1, W2, b2):
+    return rs_oracle.fc(np.maximum(rs_oracle.fc(u, W1, b1), 0), W2, b2)
+
+
+def _mlp_no_act(u, W1, b1, W2, b2):
+    return rs_oracle.fc(rs_oracle.fc(u, W1, b1), W2, b2)
+
+
+def _score_plus(h, x):
+    return np.sqrt(((h + x) ** 2).sum(axis=-1))
+
+
+def _score_residual(h, x):  # ||(h + x) - x|| = ||h||
+    return np.sqrt((h ** 2).sum(axis=-1))
+
+
+def _score_squared(h, x):
+    return ((h - x) ** 2).sum(axis=-1)
+
+
+def _score_l1(h, x):
+    return np.abs(h - x).sum(axis=-1)
+
+
+def _select_ties_high(s, k):
+    L = s.shape[0]
+    t = np.arange(1, L)
+    order = np.lexsort((-t, -s[1:]))
+    return np.concatenate([[0], np.sort(t[order[:k]])]).astype(np.int64)
+
+
+def _select_lowest(s, k):
+    L = s.shape[0]
+    t = np.arange(1, L)
+    order = np.lexsort((t, s[1:]))
+    return np.concatenate([[0], np.sort(t[order[:k]])]).astype(np.int64)
+
+
+def _select_rank_cls(s, k):
+    L = s.shape[0]
+    t = np.arange(0, L)
+    order = np.lexsort((t, -s))
+    return np.sort(t[order[: k + 1]]).astype(np.int64)
+
+
+def _select_unsorted(s, k):
+    L = s.shape[0]
+    t = np.arange(1, L)
+    order = np.lexsort((t, -s[1:]))
+    return np.concatenate([[0], t[order[:k]]]).astype(np.int64)
+
+
+def _gather_shift(y, kept):
+    return y[np.minimum(kept + 1, y.shape[0] - 1)]
+
+
+def _sublayer_score_after_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS):
+    h = rs_oracle.mlp(rs_oracle.layer_norm(x, gamma, beta, eps), W1, b1, W2, b2)
+    y = h + x
+    return h, y, rs_oracle.shift_score(y, x)
+
+
+def _sublayer_no_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS):
+    h = rs_oracle.mlp(rs_oracle.layer_norm(x, gamma, beta, eps), W1, b1, W2, b2)
+    return h, h, rs_oracle.shift_score(h, x)
+
+
+MUTATIONS = {
+    "ln_unbiased_var": ("layer_norm", _ln_unbiased),
+    "ln_drops_beta": ("layer_norm", _ln_no_beta),
+    "ln_drops_gamma": ("layer_norm", _ln_no_gamma),
+    "ln_drops_eps": ("layer_norm", _ln_no_eps),
+    "gelu_erf_without_sqrt2": ("gelu", _gelu_no_sqrt2),
+    "gelu_tanh_approx": ("gelu", _gelu_tanh),
+    "fc_transposed_weight": ("fc", _fc_transposed),
+    "fc_drops_bias": ("fc", _fc_no_bias),
+    "mlp_relu": ("mlp", _mlp_relu),
+    "mlp_no_activation": ("mlp", _mlp_no_act),
+    "score_plus_sign": ("shift_score", _score_plus),
+    "score_squared": ("shift_score", _score_squared),
+    "score_l1": ("shift_score", _score_l1),
+    "score_of_h_only": ("shift_score", _score_residual),
+    "select_ties_to_higher_index": ("select_topk", _select_ties_high),
+    "select_keeps_lowest": ("select_topk", _select_lowest),
+    "select_ranks_cls": ("select_topk", _select_rank_cls),
+    "select_unsorted_output": ("select_topk", _select_unsorted),
+    "gather_off_by_one": ("gather", _gather_shift),
+    "score_after_residual": ("sublayer", _sublayer_score_after_residual),
+    "no_residual": ("sublayer", _sublayer_no_residual),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, monkeypatch):
+    fn_name, bad = MUTATIONS[name]
+    monkeypatch.setattr(rs_oracle, fn_name, bad)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(rs_oracle)
+        except Exception as e:  # AssertionError or a shape error from a bad operand
+            caught.append((pin.__name__, type(e).__name__))
+    assert caught, f"no pin caught mutation {name}"
