@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the pruned-MLP block (LN -> fc1 -> GELU -> fc2 + residual +
+representation-shift score -> per-sample top-k -> row gather) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rs|reference]
+
+One step = one pass of the whole path over one batch of the workload (every
+stage for the chained UMT-L workload). Prints one JSON line on rank 0.
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on
+the launch stream with an L2 flush (a 256 MiB write, outside the events)
+before it; a barrier and a device synchronise on both sides of the loop; the
+max over ranks. Per-kernel durations for the roofline come from a second
+event-timed loop over the same kernels launched one step-level entry point at a
+time. `--impl reference` times the fp64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "pruned-MLP-block tokens/sec at 1 B200; % of bf16 tensor peak; select+gather GB/s"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+KERNELS_PER_STAGE = 5  # LN stats, fc1, fc2, select, gather
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.mark_start = None
+        self.mark_end = None
+        self._lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self._lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [(t, l) for t, l in self._lines
+                if self.mark_start is None or (self.mark_start <= t <= (self.mark_end or 1e30))]
+        if not rows:
+            rows = self._lines[-5:]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, l in rows:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_rate(wl, seed: int, budget_s: float):
+    """Oracle tokens/s on a bounded sample of the workload (host cores)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    inp = make_inputs(wl, seed=seed, batch=min(wl.B, 64))
+
+    def w64(w):
+        f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+        return dict(W1=f(w.W1), b1=f(w.b1), W2=f(w.W2), b2=f(w.b2), gamma=f(w.gamma),
+                    beta=f(w.beta))
+
+    weights = [w64(w) for w in inp.weights]
+    x_all = inp.x.to(torch.float64).numpy()
+    t0 = time.time()
+    done_tokens, samples = 0, 0
+    while samples < x_all.shape[0] and (time.time() - t0) < budget_s:
+        x = x_all[samples:samples + 1]
+        for s in range(wl.stages):
+            yk, _, _, _ = oracle.block_forward(x, keep_k=wl.keep_k[s], **weights[s])
+            done_tokens += x.shape[1]
+            x = yk
+        samples += 1
+    dt = time.time() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return done_tokens / dt, samples, dt, threads
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="deit_s", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline leg (0 = skip)")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args.gpus)
+    tokens_per_step = sum(wl.tokens(s) for s in range(wl.stages))
+    config = {"workload": wl.name, "B": wl.B, "L": wl.L, "C": wl.C, "H": wl.H,
+              "keep_k": list(wl.keep_k), "stages": wl.stages,
+              "tokens_per_step": tokens_per_step, "parallelism": f"replicas{world}",
+              "l2": "flushed between timed steps (256 MiB write)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        budget = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            oracle_rate(wl, 0, budget / 4)
+        rates = []
+        info = None
+        for _ in range(args.steps):
+            r, n, dt, thr = oracle_rate(wl, 0, budget)
+            rates.append(r)
+            info = (n, dt, thr)
+        v = float(np.mean(rates))
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 0,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * tokens_per_step / v, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config,
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": info[2], "kind": "oracle",
+                                 "sample": f"{info[0]} samples per step (~{info[1]:.1f} s), "
+                                           f"workload {wl.name}"},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import free_vit_token_b200 as rs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    inp = make_inputs(wl, seed=rank)
+    x = inp.x.to(dev)
+    W = [[t.to(dev) for t in (w.W1, w.b1, w.W2, w.b2, w.gamma, w.beta)] for w in inp.weights]
+    stream = torch.cuda.current_stream(dev)
+    outs = [(torch.empty(wl.B, k + 1, wl.C, dtype=torch.bfloat16, device=dev),
+             torch.empty(wl.B, k + 1, dtype=torch.int32, device=dev),
+             torch.empty(wl.B, wl.stage_L(s), dtype=torch.float32, device=dev))
+            for s, k in enumerate(wl.keep_k)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(x0):
+        xs = x0
+        for s, k in enumerate(wl.keep_k):
+            rs.rs_block_forward(xs, *W[s], k, *outs[s], stream=stream)
+            xs = outs[s][0]
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(x)
+    torch.cuda.synchronize()
+    assert rs.rs_get_last_device_error() == 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark_start = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(x)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.mark_end = time.time()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    status = rs.rs_get_last_device_error()
+    assert status == 0, rs.status_string(status)
+    ms_per_step = total_ms / args.steps
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # ---- per-kernel breakdown (same kernels, one step-level entry point at a time)
+    kt = {"fc1": [], "fc2": [], "select": [], "gather": []}
+    M0 = wl.tokens(0)
+    hid = torch.empty(M0 * wl.H, dtype=torch.bfloat16, device=dev)
+    ybuf = torch.empty(M0 * wl.C, dtype=torch.bfloat16, device=dev)
+    np_ = rs.rs_num_partials(wl.C)
+    pbuf = torch.empty(M0 * np_, dtype=torch.float32, device=dev)
+    nrep = max(10, min(args.steps, 200))
+    recs = []
+    for i in range(nrep):
+        flush.zero_()
+        xs = x
+        for s, k in enumerate(wl.keep_k):
+            L_s = wl.stage_L(s)
+            M = wl.B * L_s
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            x2 = xs.reshape(M, wl.C)
+            h2 = hid[: M * wl.H].view(M, wl.H)
+            y2 = ybuf[: M * wl.C].view(M, wl.C)
+            p2 = pbuf[: M * np_].view(M, np_)
+            e[0].record(stream)
+            rs.rs_ln_fc1_gelu(x2, W[s][0], W[s][1], W[s][4], W[s][5], hidden=h2, stream=stream)
+            e[1].record(stream)
+            rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
+            e[2].record(stream)
+            rs.rs_select_topk(p2, wl.B, L_s, k, scores=outs[s][2], kept_idx=outs[s][1],
+                              stream=stream)
+            e[3].record(stream)
+            rs.rs_gather_rows(y2.view(wl.B, L_s, wl.C), outs[s][1], k, y_kept=outs[s][0],
+                              stream=stream)
+            e[4].record(stream)
+            recs.append((s, e))
+            xs = outs[s][0]
+    torch.cuda.synchronize()
+    per_stage = {}
+    for s, e in recs:
+        d = per_stage.setdefault(s, {"fc1": [], "fc2": [], "select": [], "gather": []})
+        d["fc1"].append(e[0].elapsed_time(e[1]))
+        d["fc2"].append(e[1].elapsed_time(e[2]))
+        d["select"].append(e[2].elapsed_time(e[3]))
+        d["gather"].append(e[3].elapsed_time(e[4]))
+    gemm_flops = {s: 2.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages)}
+    fc_ms = {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage) for n in ("fc1", "fc2")}
+    dominant = max(fc_ms, key=fc_ms.get)
+    flops = sum(gemm_flops.values())
+    achieved_tf = flops / (fc_ms[dominant] / 1e3) / 1e12
+    sel_ms = sum(statistics.mean(per_stage[s]["select"]) + statistics.mean(per_stage[s]["gather"])
+                 for s in per_stage)
+    sg_bytes = 0
+    for s, k in enumerate(wl.keep_k):
+        M = wl.tokens(s)
+        sg_bytes += M * np_ * 4 + M * 4 + wl.B * (k + 1) * 4       # select: partials in, scores + idx out
+        sg_bytes += wl.B * (k + 1) * (4 + 2 * wl.C * 2)           # gather: idx in, rows in + out
+    sg_gbs = sg_bytes / (sel_ms / 1e3) / 1e9
+    block_flops = sum(4.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages))
+
+    # ---- end to end through the public call with host buffers
+    x_h = inp.x.pin_memory()
+    h2d = x_h.numel() * x_h.element_size()
+    outs_h = [tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs[-1])]
+    d2h = sum(o.numel() * o.element_size() for o in outs_h[0])
+    x_d = torch.empty_like(x)
+    n_e2e = max(5, min(args.steps, 100))
+    e2e_ev = []
+    barrier(world)
+    for i in range(n_e2e):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x_d.copy_(x_h, non_blocking=True)
+        step(x_d)
+        for oh, od in zip(outs_h[0], outs[-1]):
+            oh.copy_(od, non_blocking=True)
+        b.record(stream)
+        e2e_ev.append((a, b))
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world) / n_e2e
+    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+    clocks.stop()
+
+    cpu = None
+    if rank == 0 and args.cpu_budget > 0:
+        r, n, dt, thr = oracle_rate(wl, 0, args.cpu_budget)
+        cpu = {"value": r, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": f"{n} of {wl.B} samples of {wl.name} (all stages) in {dt:.1f} s "
+                         f"on the host, fp64 numpy/BLAS"}
+
+    peak_tf = peaks["bf16"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "tensor", "kernel": f"{dominant} (tcgen05 GEMM)",
+                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved_tf / peak_tf, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "kernel_ms": fc_ms[dominant]},
+        "block_tflops": block_flops / (ms_per_step / 1e3) / 1e12,
+        "block_frac_of_bf16_peak": block_flops / (ms_per_step / 1e3) / 1e12 / peak_tf,
+        "kernel_ms": {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage)
+                      for n in ("fc1", "fc2", "select", "gather")},
+        "select_gather": {"GBps": sg_gbs, "frac_hbm": sg_gbs / peaks["hbm"],
+                          "bytes": sg_bytes, "ms": sel_ms},
+        "images_per_s": world * wl.B / (ms_per_step / 1e3),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_STAGE * wl.stages * args.steps,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    rs.rs_release_workspace()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,20 @@
+"""B200 (sm_100a) implementation of the pruned-MLP block of Representation Shift.
+
+The compute lives in ``librs.so`` (CUDA kernels behind a C ABI, include/rs.h);
+``free_vit_token_b200.rs`` is its ctypes binding.
+"""
+from .rs import (  # noqa: F401
+    RsError,
+    lib,
+    rs_block_forward,
+    rs_fc2_residual_shift,
+    rs_gather_rows,
+    rs_get_last_device_error,
+    rs_ln_fc1_gelu,
+    rs_ln_stats,
+    rs_num_partials,
+    rs_release_workspace,
+    rs_select_topk,
+    rs_workspace_bytes,
+    status_string,
+)

@@ -1,0 +1,361 @@
+// rs_api.cu -- the C ABI of librs.so (declared and documented in include/rs.h):
+// argument validation, the per-device workspace, TMA tensor maps and the launch
+// sequence of the pruned-MLP block of "Representation Shift: Unifying Token
+// Compression with FlashAttention" (§3.3 Eq. (6), §3.2 Eq. (4), §3.1 pruning).
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "rs.h"
+#include "rs_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DevState {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* err = nullptr;  // device status flag (one int)
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DevState g_dev[kMaxDevices];
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t stats, hidden, y, partials, total;
+};
+
+WsLayout ws_layout(int64_t M, int C, int H) {
+  WsLayout w{};
+  size_t off = 0;
+  w.stats = off;
+  off = align_up(off + static_cast<size_t>(M) * 8, 1024);
+  w.hidden = off;
+  off = align_up(off + static_cast<size_t>(M) * H * 2, 1024);
+  w.y = off;
+  off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
+  w.partials = off;
+  off = align_up(off + static_cast<size_t>(M) * (2 * C / rs::fc2_block_n(C)) * 4, 1024);
+  w.total = off;
+  return w;
+}
+
+// Caller holds g_mu.
+int dev_state(DevState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RS_ERR_CUDA;
+  DevState& st = g_dev[dev];
+  if (st.err == nullptr) {
+    if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return RS_ERR_CUDA;
+    int* e = nullptr;
+    if (cudaMalloc(&e, 256) != cudaSuccess) return RS_ERR_NO_MEM;
+    if (cudaMemset(e, 0, 256) != cudaSuccess) return RS_ERR_CUDA;
+    st.err = e;
+  }
+  *out = &st;
+  return RS_OK;
+}
+
+// Caller holds g_mu.
+int ensure_ws(DevState& st, size_t bytes) {
+  if (st.ws_bytes >= bytes) return RS_OK;
+  if (st.ws != nullptr) {
+    cudaDeviceSynchronize();
+    cudaFree(st.ws);
+    st.ws = nullptr;
+    st.ws_bytes = 0;
+  }
+  if (cudaMalloc(&st.ws, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    st.ws = nullptr;
+    return RS_ERR_NO_MEM;
+  }
+  st.ws_bytes = bytes;
+  return RS_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 [rows, inner] viewed as tiles of {64 elements, box_rows rows},
+// 128-byte swizzled in shared memory; rows past the end read as zero.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return RS_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RS_OK : RS_ERR_CUDA;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool al8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+bool al4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_width(int C) {
+  return (C < 64 || C > RS_MAX_C || C % 64 != 0) ? RS_ERR_SHAPE : RS_OK;
+}
+int check_hidden(int H) {
+  return (H < 64 || H > RS_MAX_H || H % 64 != 0) ? RS_ERR_SHAPE : RS_OK;
+}
+int check_rows(int64_t M, int C, int H) {
+  if (M < 0) return RS_ERR_SHAPE;
+  const int64_t w = C > H ? C : H;
+  return (M * w >= (static_cast<int64_t>(1) << 31)) ? RS_ERR_SHAPE : RS_OK;
+}
+
+#define RS_TRY(expr)              \
+  do {                            \
+    const int _s = (expr);        \
+    if (_s != RS_OK) return _s;   \
+  } while (0)
+#define RS_CUDA(expr)                                       \
+  do {                                                      \
+    if ((expr) != cudaSuccess) {                            \
+      cudaGetLastError();                                   \
+      return RS_ERR_CUDA;                                   \
+    }                                                       \
+  } while (0)
+
+int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, const void* b1,
+            const void* gamma, const void* beta, float* stats, void* hidden, cudaStream_t s) {
+  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, s));
+  const int bn = rs::fc1_block_n(H);
+  CUtensorMap tmX, tmW;
+  RS_TRY(make_tmap(&tmX, x, C, M, 128));
+  RS_TRY(make_tmap(&tmW, W1, C, H, bn));
+  rs::MlpParams p{};
+  p.M = M;
+  p.N = H;
+  p.K = C;
+  p.n_blocks = H / bn;
+  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.ln_gamma = static_cast<const __nv_bfloat16*>(gamma);
+  p.ln_beta = static_cast<const __nv_bfloat16*>(beta);
+  p.stats = reinterpret_cast<const float2*>(stats);
+  p.bias = static_cast<const __nv_bfloat16*>(b1);
+  p.out = static_cast<__nv_bfloat16*>(hidden);
+  p.err = st.err;
+  p.timeout_ns = rs::kDefaultTimeoutNs;
+  RS_CUDA(rs::launch_fc1(tmX, tmW, p, bn, st.num_sms, s));
+  return RS_OK;
+}
+
+int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H, const void* W2,
+            const void* b2, void* y, float* partials, cudaStream_t s) {
+  const int bn = rs::fc2_block_n(C);
+  CUtensorMap tmH, tmW;
+  RS_TRY(make_tmap(&tmH, hidden, H, M, 128));
+  RS_TRY(make_tmap(&tmW, W2, H, C, bn));
+  rs::MlpParams p{};
+  p.M = M;
+  p.N = C;
+  p.K = H;
+  p.n_blocks = C / bn;
+  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.bias = static_cast<const __nv_bfloat16*>(b2);
+  p.out = static_cast<__nv_bfloat16*>(y);
+  p.resid = static_cast<const __nv_bfloat16*>(x);
+  p.partials = partials;
+  p.num_partials = 2 * p.n_blocks;
+  p.err = st.err;
+  p.timeout_ns = rs::kDefaultTimeoutNs;
+  RS_CUDA(rs::launch_fc2(tmH, tmW, p, bn, st.num_sms, s));
+  return RS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rs_status_string(int status) {
+  switch (status) {
+    case RS_OK: return "RS_OK";
+    case RS_ERR_NULL: return "RS_ERR_NULL: a required pointer is NULL";
+    case RS_ERR_SHAPE: return "RS_ERR_SHAPE: B, L, C or H outside the supported limits";
+    case RS_ERR_KEEP_K: return "RS_ERR_KEEP_K: keep_k outside 0..L-1";
+    case RS_ERR_ALIGN: return "RS_ERR_ALIGN: a pointer is not suitably aligned";
+    case RS_ERR_CUDA: return "RS_ERR_CUDA: the CUDA runtime or driver reported an error";
+    case RS_ERR_DEVICE_TIMEOUT: return "RS_ERR_DEVICE_TIMEOUT: a kernel pipeline wait timed out";
+    case RS_ERR_NO_MEM: return "RS_ERR_NO_MEM: workspace allocation failed";
+    default: return "unknown rs_status";
+  }
+}
+
+int rs_num_partials(int C) { return check_width(C) == RS_OK ? 2 * C / rs::fc2_block_n(C) : 0; }
+
+uint64_t rs_workspace_bytes(int B, int L, int C, int H) {
+  if (B < 0 || L < 1 || check_width(C) != RS_OK || check_hidden(H) != RS_OK) return 0;
+  return ws_layout(static_cast<int64_t>(B) * L, C, H).total;
+}
+
+int rs_ln_stats(const void* x, int M, int C, float* stats, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_rows(M, C, C));
+  if (M == 0) return RS_OK;
+  if (!x || !stats) return RS_ERR_NULL;
+  if (!al16(x) || !al8(stats)) return RS_ERR_ALIGN;
+  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                   const void* gamma, const void* beta, void* hidden, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (M == 0) return RS_OK;
+  if (!x || !W1 || !b1 || !gamma || !beta || !hidden) return RS_ERR_NULL;
+  if (!al16(x) || !al16(W1) || !al16(b1) || !al16(gamma) || !al16(beta) || !al16(hidden))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  RS_TRY(ensure_ws(*st, align_up(static_cast<size_t>(M) * 8, 1024)));
+  return run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, static_cast<float*>(st->ws), hidden,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H, const void* W2,
+                          const void* b2, void* y, float* partials, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (M == 0) return RS_OK;
+  if (!hidden || !x || !W2 || !b2 || !y || !partials) return RS_ERR_NULL;
+  if (!al16(hidden) || !al16(x) || !al16(W2) || !al16(b2) || !al16(y) || !al4(partials))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, static_cast<cudaStream_t>(stream));
+}
+
+int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
+                   float* scores, int32_t* kept_idx, void* stream) {
+  if (B < 0 || L < 1 || L > RS_MAX_L || num_partials < 1 || num_partials > 64)
+    return RS_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * L * num_partials >= (static_cast<int64_t>(1) << 31))
+    return RS_ERR_SHAPE;
+  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  if (B == 0) return RS_OK;
+  if (!partials || !scores || !kept_idx) return RS_ERR_NULL;
+  if (!al4(partials) || !al4(scores) || !al4(kept_idx)) return RS_ERR_ALIGN;
+  RS_CUDA(rs::launch_select(partials, num_partials, B, L, keep_k, scores, kept_idx,
+                            static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
+                   void* y_kept, void* stream) {
+  RS_TRY(check_width(C));
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, C));
+  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  if (B == 0) return RS_OK;
+  if (!y || !kept_idx || !y_kept) return RS_ERR_NULL;
+  if (!al16(y) || !al4(kept_idx) || !al16(y_kept)) return RS_ERR_ALIGN;
+  int num_sms = 148;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevState* st = nullptr;
+    RS_TRY(dev_state(&st));
+    num_sms = st->num_sms;
+  }
+  RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k, y_kept, num_sms,
+                            static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, const void* b1,
+                     const void* W2, const void* b2, const void* gamma, const void* beta,
+                     int keep_k, void* y_kept, int32_t* kept_idx, float* scores, void* stream) {
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  const int64_t M64 = static_cast<int64_t>(B) * L;
+  RS_TRY(check_rows(M64, C, H));
+  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  if (B == 0) return RS_OK;
+  if (!x || !W1 || !b1 || !W2 || !b2 || !gamma || !beta || !y_kept || !kept_idx || !scores)
+    return RS_ERR_NULL;
+  if (!al16(x) || !al16(W1) || !al16(b1) || !al16(W2) || !al16(b2) || !al16(gamma) ||
+      !al16(beta) || !al16(y_kept) || !al4(kept_idx) || !al4(scores))
+    return RS_ERR_ALIGN;
+  const int M = static_cast<int>(M64);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  const WsLayout w = ws_layout(M, C, H);
+  RS_TRY(ensure_ws(*st, w.total));
+  uint8_t* ws = static_cast<uint8_t*>(st->ws);
+  float* stats = reinterpret_cast<float*>(ws + w.stats);
+  void* hidden = ws + w.hidden;
+  void* y = ws + w.y;
+  float* partials = reinterpret_cast<float*>(ws + w.partials);
+  const int np = 2 * C / rs::fc2_block_n(C);
+
+  RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, stats, hidden, s));
+  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s));
+  RS_CUDA(rs::launch_select(partials, np, B, L, keep_k, scores, kept_idx, s));
+  RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k, y_kept, st->num_sms, s));
+  return RS_OK;
+}
+
+int rs_get_last_device_error(void* stream) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return RS_ERR_CUDA;
+  }
+  int v = 0;
+  RS_CUDA(cudaMemcpy(&v, st->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) RS_CUDA(cudaMemset(st->err, 0, sizeof(int)));
+  return v;
+}
+
+void rs_release_workspace(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    DevState& st = g_dev[d];
+    if (st.ws == nullptr) continue;
+    if (cudaSetDevice(d) == cudaSuccess) {
+      cudaDeviceSynchronize();
+      cudaFree(st.ws);
+    }
+    st.ws = nullptr;
+    st.ws_bytes = 0;
+  }
+  cudaSetDevice(cur);
+}
+
+}  // extern "C"

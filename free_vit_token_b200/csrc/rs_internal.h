@@ -1,0 +1,48 @@
+// rs_internal.h -- declarations shared by the library's translation units
+// (kernel parameter blocks and host-side launchers). Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rs.h"
+
+namespace rs {
+
+constexpr float kLnEps = 1e-6f;          // LayerNorm epsilon (the pages do not state one)
+constexpr int kEpiGelu = 0;              // fc1 epilogue: + b1, erf-GELU, bf16 store
+constexpr int kEpiResidShift = 1;        // fc2 epilogue: + b2, residual, shift partials
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // one pipeline wait: 4 s
+
+struct MlpParams {
+  int M, N, K;                    // output rows, output columns, reduction length
+  int n_blocks, num_tiles;        // N / BN, ceil(M / 128) * n_blocks
+  const __nv_bfloat16* ln_gamma;  // [K]   fc1 only
+  const __nv_bfloat16* ln_beta;   // [K]   fc1 only
+  const float2* stats;            // [M]   fc1 only: (mean, rstd) per row
+  const __nv_bfloat16* bias;      // [N]
+  __nv_bfloat16* out;             // [M, N] hidden (fc1) or y (fc2)
+  const __nv_bfloat16* resid;     // [M, N] x' (fc2 only)
+  float* partials;                // [M, num_partials] (fc2 only)
+  int num_partials;               // 2 * n_blocks (fc2)
+  int* err;                       // device status flag
+  unsigned long long timeout_ns;  // limit of one pipeline wait
+};
+
+size_t mlp_smem_bytes(int bn, bool ln, int K);
+int fc1_block_n(int H);
+int fc2_block_n(int C);
+cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, cudaStream_t stream);
+cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const MlpParams& p, int bn,
+                       int num_sms, cudaStream_t s);
+cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p,
+                       int bn, int num_sms, cudaStream_t s);
+cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
+                          float* scores, int32_t* kept_idx, cudaStream_t stream);
+cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
+                          void* y_kept, int num_sms, cudaStream_t stream);
+
+}  // namespace rs

@@ -1,0 +1,188 @@
+"""ctypes binding of librs.so (see include/rs.h): argument marshalling only.
+
+Every function here forwards torch tensors' device pointers and sizes to the C
+entry point of the same name and raises ``RsError`` on a non-zero status. All
+arithmetic runs in the library's CUDA kernels; there is no other code path, and
+a missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librs.so")
+
+RS_OK = 0
+RS_ERR_NULL = 1
+RS_ERR_SHAPE = 2
+RS_ERR_KEEP_K = 3
+RS_ERR_ALIGN = 4
+RS_ERR_CUDA = 5
+RS_ERR_DEVICE_TIMEOUT = 6
+RS_ERR_NO_MEM = 7
+
+_vp, _i, _fp, _ip = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+SIGNATURES = {
+    "rs_block_forward": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _ip,
+                              _fp, _vp]),
+    "rs_ln_stats": (_i, [_vp, _i, _i, _fp, _vp]),
+    "rs_ln_fc1_gelu": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
+    "rs_num_partials": (_i, [_i]),
+    "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
+    "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
+    "rs_status_string": (ctypes.c_char_p, [_i]),
+    "rs_get_last_device_error": (_i, [_vp]),
+    "rs_release_workspace": (None, []),
+    "rs_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),
+}
+
+_lib = None
+
+
+class RsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded librs.so. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m free_vit_token_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().rs_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != RS_OK:
+        raise RsError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return t.data_ptr() or None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream or None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream or None
+    return int(stream) or None
+
+
+def rs_block_forward(x: torch.Tensor, W1, b1, W2, b2, gamma, beta, keep_k: int,
+                     y_kept: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
+                     scores: Optional[torch.Tensor] = None, stream=None
+                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """x [B, L, C] bf16 -> (y_kept [B, 1+k, C] bf16, kept_idx [B, 1+k] int32, scores [B, L] fp32)."""
+    B, L, C = x.shape
+    H = W1.shape[0]
+    dev = x.device
+    if y_kept is None:
+        y_kept = torch.empty(B, keep_k + 1, C, dtype=torch.bfloat16, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
+    if scores is None:
+        scores = torch.empty(B, L, dtype=torch.float32, device=dev)
+    st = lib().rs_block_forward(_ptr(x), B, L, C, H, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                                _ptr(gamma), _ptr(beta), int(keep_k), _ptr(y_kept),
+                                _ptr(kept_idx), _ptr(scores), _stream(stream))
+    _check(st, "rs_block_forward")
+    return y_kept, kept_idx, scores
+
+
+def rs_ln_stats(x2d: torch.Tensor, stats: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, C = x2d.shape
+    if stats is None:
+        stats = torch.empty(M, 2, dtype=torch.float32, device=x2d.device)
+    _check(lib().rs_ln_stats(_ptr(x2d), M, C, _ptr(stats), _stream(stream)), "rs_ln_stats")
+    return stats
+
+
+def rs_ln_fc1_gelu(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    M, C = x2d.shape
+    H = W1.shape[0]
+    if hidden is None:
+        hidden = torch.empty(M, H, dtype=torch.bfloat16, device=x2d.device)
+    st = lib().rs_ln_fc1_gelu(_ptr(x2d), M, C, H, _ptr(W1), _ptr(b1), _ptr(gamma), _ptr(beta),
+                              _ptr(hidden), _stream(stream))
+    _check(st, "rs_ln_fc1_gelu")
+    return hidden
+
+
+def rs_num_partials(C: int) -> int:
+    return int(lib().rs_num_partials(int(C)))
+
+
+def rs_fc2_residual_shift(hidden: torch.Tensor, x2d: torch.Tensor, W2, b2,
+                          y: Optional[torch.Tensor] = None, partials: Optional[torch.Tensor] = None,
+                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    M, H = hidden.shape
+    C = x2d.shape[1]
+    if y is None:
+        y = torch.empty(M, C, dtype=torch.bfloat16, device=x2d.device)
+    if partials is None:
+        partials = torch.empty(M, rs_num_partials(C), dtype=torch.float32, device=x2d.device)
+    st = lib().rs_fc2_residual_shift(_ptr(hidden), _ptr(x2d), M, C, H, _ptr(W2), _ptr(b2), _ptr(y),
+                                     _ptr(partials), _stream(stream))
+    _check(st, "rs_fc2_residual_shift")
+    return y, partials
+
+
+def rs_select_topk(partials: torch.Tensor, B: int, L: int, keep_k: int,
+                   scores: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    P = partials.shape[-1]
+    dev = partials.device
+    if scores is None:
+        scores = torch.empty(B, L, dtype=torch.float32, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
+    st = lib().rs_select_topk(_ptr(partials), P, B, L, int(keep_k), _ptr(scores), _ptr(kept_idx),
+                              _stream(stream))
+    _check(st, "rs_select_topk")
+    return scores, kept_idx
+
+
+def rs_gather_rows(y: torch.Tensor, kept_idx: torch.Tensor, keep_k: int,
+                   y_kept: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    B, L, C = y.shape
+    if y_kept is None:
+        y_kept = torch.empty(B, keep_k + 1, C, dtype=y.dtype, device=y.device)
+    st = lib().rs_gather_rows(_ptr(y), B, L, C, _ptr(kept_idx), int(keep_k), _ptr(y_kept),
+                              _stream(stream))
+    _check(st, "rs_gather_rows")
+    return y_kept
+
+
+def rs_get_last_device_error(stream=None) -> int:
+    return int(lib().rs_get_last_device_error(_stream(stream)))
+
+
+def rs_release_workspace() -> None:
+    lib().rs_release_workspace()
+
+
+def rs_workspace_bytes(B: int, L: int, C: int, H: int) -> int:
+    return int(lib().rs_workspace_bytes(B, L, C, H))

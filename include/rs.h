@@ -1,0 +1,150 @@
+/*
+ * rs.h -- C ABI of librs.so: the pruned-MLP block of Representation Shift on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "Representation Shift: Unifying Token Compression with
+ * FlashAttention" (arXiv 2508.00367v1, ICCV 2025).
+ *   - Block, §3.3 Eq. (6):      y = x-hat = MLP(LN(x')) + x'
+ *   - Score, §3.2 Eq. (4) with F = MLP (§3.3 "Operation choice" (ii)) and
+ *     D = L2 (§3.3 "Distance metrics" (i)):   s = || MLP(LN(x')) - x' ||_2
+ *   - Pruning, §3.1 / §3.2: drop the lowest-s tokens, keep x-tilde in
+ *     R^{(N-r) x C} for the attention layer that follows.
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor argument is a DEVICE pointer owned by the caller, contiguous,
+ *     row-major, 16-byte aligned unless stated otherwise. "bf16" is IEEE
+ *     bfloat16 (torch.bfloat16). Nothing here frees or keeps caller memory.
+ *   - Weights use the nn.Linear layout: W1 is [H, C], W2 is [C, H].
+ *   - Token rows are [B, L, C] with r = b*L + t; t = 0 is the CLS token and
+ *     t = 1..L-1 are patch tokens.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Every call is asynchronous on that stream and never synchronises,
+ *     except rs_get_last_device_error and rs_release_workspace.
+ *   - Return value: an rs_status. Argument errors are detected on the host and
+ *     returned before anything is launched; outputs are then left untouched.
+ *     RS_ERR_CUDA reports a launch or allocation failure from the CUDA runtime.
+ *   - Device-side failures (a pipeline wait that ran past its time limit) do
+ *     not trap: the kernel records RS_ERR_DEVICE_TIMEOUT in a device flag,
+ *     drains its own work and returns; rs_get_last_device_error reports it.
+ *   - Shape limits: 1 <= L <= RS_MAX_L; C and H multiples of 64 with
+ *     64 <= C <= RS_MAX_C and 64 <= H <= RS_MAX_H; 0 <= keep_k <= L-1;
+ *     B*L*max(C,H) < 2^31. B = 0 is an empty batch: RS_OK, nothing launched.
+ *   - Library workspace: rs_block_forward and the fc steps use a per-device
+ *     workspace owned by the library (cudaMalloc'd on first use, grown on
+ *     demand, reused across calls). Growing it synchronises the device. Calls
+ *     that share a device must be ordered on one stream (they share it).
+ */
+#ifndef RS_H_
+#define RS_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RS_MAX_L 16384
+#define RS_MAX_C 2048
+#define RS_MAX_H 16384
+
+typedef enum rs_status {
+  RS_OK = 0,
+  RS_ERR_NULL = 1,            /* a required pointer is NULL */
+  RS_ERR_SHAPE = 2,           /* B, L, C or H outside the limits above */
+  RS_ERR_KEEP_K = 3,          /* keep_k outside 0..L-1 */
+  RS_ERR_ALIGN = 4,           /* a pointer is not 16-byte (tensors) / 4-byte (int, float) aligned */
+  RS_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */
+  RS_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up waiting on its pipeline (device flag) */
+  RS_ERR_NO_MEM = 7           /* the workspace could not be allocated */
+} rs_status;
+
+/*
+ * rs_block_forward -- the whole hot path for one block (Eq. (6) + Eq. (4) +
+ * pruning), on `stream`:
+ *   u   = LN(x')            per row: (x'-mean)/sqrt(var+1e-6)*gamma+beta,
+ *                           biased variance
+ *   h   = W2 GELU(W1 u + b1) + b2   (exact erf GELU; fp32 accumulation of bf16
+ *                                    operands; the hidden activation is
+ *                                    rounded to bf16 between fc1 and fc2)
+ *   y   = x' + h            (rounded to bf16)
+ *   s_t = || h_t - x'_t ||_2 (h in fp32, before rounding)
+ *   kept_idx[b] = [0] ++ ascending(the keep_k patch tokens of largest s;
+ *                 equal s -> lower t first)
+ *   y_kept[b, j, :] = y[b, kept_idx[b, j], :]
+ *
+ *   x        [B, L, C] bf16   input x' (the attention sublayer's output)
+ *   W1 [H, C], b1 [H], W2 [C, H], b2 [C], gamma [C], beta [C]: bf16
+ *   keep_k   patch tokens kept per sample (CLS is kept in addition)
+ *   y_kept   [B, 1+keep_k, C] bf16   output
+ *   kept_idx [B, 1+keep_k] int32     output (4-byte aligned)
+ *   scores   [B, L] fp32             output, every token incl. CLS (4-byte aligned)
+ */
+int rs_block_forward(const void* x, int B, int L, int C, int H,
+                     const void* W1, const void* b1, const void* W2, const void* b2,
+                     const void* gamma, const void* beta, int keep_k,
+                     void* y_kept, int32_t* kept_idx, float* scores, void* stream);
+
+/*
+ * Step-level entry points. rs_block_forward launches exactly these kernels in
+ * this order; they are exported so that each step can be checked on its own.
+ */
+
+/* LayerNorm row statistics (Eq. (6)'s LN, the reduction half):
+ * stats[2r] = mean of x'[r, :], stats[2r+1] = 1/sqrt(biased var + 1e-6).
+ * x [M, C] bf16; stats [M, 2] fp32 (8-byte aligned). */
+int rs_ln_stats(const void* x, int M, int C, float* stats, void* stream);
+
+/* a = GELU(LN(x') W1^T + b1) as bf16 [M, H], the LN applied while staging
+ * fc1's A operand (uses rs_ln_stats internally; its stats live in the
+ * library workspace). x [M, C]; hidden [M, H] bf16 output. */
+int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                   const void* gamma, const void* beta, void* hidden, void* stream);
+
+/* fc2 with the residual and the shift partials (Eq. (6) and Eq. (4)):
+ *   h = hidden W2^T + b2 (fp32), y = bf16(x' + h) [M, C],
+ *   partials[r, j] = sum over column group j of (h[r,c] - x'[r,c])^2 (fp32).
+ * partials is [M, rs_num_partials(C)] fp32; summing a row's partials left to
+ * right gives s_t^2. */
+int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H,
+                          const void* W2, const void* b2, void* y, float* partials,
+                          void* stream);
+
+/* Number of per-row partial sums rs_fc2_residual_shift writes for width C
+ * (0 if C is unsupported). */
+int rs_num_partials(int C);
+
+/* Score finalisation and per-sample top-k (§3.2 drop the lowest-k scores):
+ *   scores[b, t] = sqrt(sum_{j=0..P-1} partials[b*L+t, j])  (fp32, left to right)
+ *   kept_idx[b]  = [0] ++ ascending(top keep_k of t = 1..L-1 by score; ties to
+ *                  the lower t). Selection compares the fp32 score bits.
+ * partials [B*L, P] fp32 with 1 <= P <= 64; scores [B, L]; kept_idx [B, 1+keep_k]. */
+int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
+                   float* scores, int32_t* kept_idx, void* stream);
+
+/* Row gather, the pruned set x-tilde (§3.1):
+ * y_kept[b, j, :] = y[b, kept_idx[b, j], :]. y [B, L, C] bf16; kept_idx
+ * [B, 1+keep_k] int32 with entries in 0..L-1 (not checked on the device);
+ * y_kept [B, 1+keep_k, C] bf16. */
+int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
+                   void* y_kept, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* rs_status_string(int status);
+
+/* Synchronises `stream`, returns and clears the current device's flag
+ * (RS_OK or RS_ERR_DEVICE_TIMEOUT), or RS_ERR_CUDA if the synchronisation
+ * itself failed. */
+int rs_get_last_device_error(void* stream);
+
+/* Frees the library workspace of every device (synchronises each device that
+ * has one). The next call that needs it allocates it again. */
+void rs_release_workspace(void);
+
+/* Bytes of workspace rs_block_forward needs for these sizes (0 if invalid). */
+uint64_t rs_workspace_bytes(int B, int L, int C, int H);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RS_H_ */

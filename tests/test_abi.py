@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before launching anything (no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_vit_token_b200.rs as rs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # 16-byte aligned fake device address: never dereferenced on these paths
+MIS = 0x10002   # misaligned fake address
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "rs.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rs_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "rs_block_forward" in names and len(names) >= 10
+    lib = rs.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(rs.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings():
+    for code in range(8):
+        assert rs.status_string(code).startswith("RS_")
+    assert "unknown" in rs.status_string(99)
+
+
+def test_num_partials_and_workspace():
+    assert rs.rs_num_partials(384) == 4      # two 192-wide column groups, two halves each
+    assert rs.rs_num_partials(768) == 6
+    assert rs.rs_num_partials(1024) == 8
+    assert rs.rs_num_partials(192) == 2
+    assert rs.rs_num_partials(100) == 0
+    wb = rs.rs_workspace_bytes(256, 197, 384, 1536)
+    M = 256 * 197
+    assert wb >= M * 1536 * 2 + M * 384 * 2 + M * 8 + M * 4 * 4
+    assert rs.rs_workspace_bytes(1, 1, 65, 64) == 0
+
+
+def _fwd(x=FAKE, B=2, L=197, C=192, H=768, w=FAKE, keep_k=137, out=FAKE, idx=FAKE, sc=FAKE):
+    return rs.lib().rs_block_forward(x, B, L, C, H, w, w, w, w, w, w, keep_k, out, idx, sc, None)
+
+
+def test_block_forward_argument_errors():
+    assert _fwd(B=0) == rs.RS_OK                  # empty batch: nothing to do
+    assert _fwd(B=0, x=None, out=None) == rs.RS_OK
+    assert _fwd(x=None) == rs.RS_ERR_NULL
+    assert _fwd(w=None) == rs.RS_ERR_NULL
+    assert _fwd(idx=None) == rs.RS_ERR_NULL
+    assert _fwd(B=-1) == rs.RS_ERR_SHAPE
+    assert _fwd(L=0) == rs.RS_ERR_SHAPE
+    assert _fwd(L=16385, keep_k=1) == rs.RS_ERR_SHAPE
+    assert _fwd(C=200) == rs.RS_ERR_SHAPE
+    assert _fwd(C=4096) == rs.RS_ERR_SHAPE
+    assert _fwd(H=100) == rs.RS_ERR_SHAPE
+    assert _fwd(B=1 << 20, C=2048, H=2048, L=1024) == rs.RS_ERR_SHAPE
+    assert _fwd(keep_k=-1) == rs.RS_ERR_KEEP_K
+    assert _fwd(keep_k=197) == rs.RS_ERR_KEEP_K
+    assert _fwd(x=MIS) == rs.RS_ERR_ALIGN
+    assert _fwd(out=MIS) == rs.RS_ERR_ALIGN
+    assert _fwd(idx=FAKE + 1) == rs.RS_ERR_ALIGN
+
+
+def test_step_entry_points_argument_errors():
+    L = rs.lib()
+    assert L.rs_ln_stats(None, 10, 192, FAKE, None) == rs.RS_ERR_NULL
+    assert L.rs_ln_stats(FAKE, 10, 100, FAKE, None) == rs.RS_ERR_SHAPE
+    assert L.rs_ln_stats(FAKE, 0, 192, FAKE, None) == rs.RS_OK
+    assert L.rs_ln_fc1_gelu(FAKE, 10, 192, 770, FAKE, FAKE, FAKE, FAKE, FAKE, None) == rs.RS_ERR_SHAPE
+    assert L.rs_ln_fc1_gelu(FAKE, 10, 192, 768, None, FAKE, FAKE, FAKE, FAKE, None) == rs.RS_ERR_NULL
+    assert L.rs_ln_fc1_gelu(MIS, 10, 192, 768, FAKE, FAKE, FAKE, FAKE, FAKE, None) == rs.RS_ERR_ALIGN
+    assert L.rs_fc2_residual_shift(FAKE, FAKE, 10, 192, 768, FAKE, FAKE, FAKE, None, None) == rs.RS_ERR_NULL
+    assert L.rs_select_topk(FAKE, 0, 2, 10, 3, FAKE, FAKE, None) == rs.RS_ERR_SHAPE
+    assert L.rs_select_topk(FAKE, 4, 2, 10, 10, FAKE, FAKE, None) == rs.RS_ERR_KEEP_K
+    assert L.rs_select_topk(FAKE, 4, 0, 10, 3, None, None, None) == rs.RS_OK
+    assert L.rs_select_topk(FAKE, 4, 2, 10, 3, FAKE, FAKE + 2, None) == rs.RS_ERR_ALIGN
+    assert L.rs_gather_rows(FAKE, 2, 10, 192, FAKE, 10, FAKE, None) == rs.RS_ERR_KEEP_K
+    assert L.rs_gather_rows(FAKE, 2, 10, 192, None, 3, FAKE, None) == rs.RS_ERR_NULL
+
+
+def test_library_has_no_torch_or_libcuda_link_dependency():
+    out = os.popen(f"ldd {rs.LIB_PATH}").read()
+    assert "libtorch" not in out and "libc10" not in out

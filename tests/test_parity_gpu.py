@@ -1,0 +1,240 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from workloads import WORKLOADS, make_inputs, random_block, random_partials
+
+pytestmark = pytest.mark.gpu
+
+dev = torch.device("cuda:0")
+
+
+def _rs():
+    import free_vit_token_b200 as rs  # deferred: collection must not need a GPU
+    return rs
+
+
+def _to_dev(w):
+    return [t.to(dev) for t in (w.W1, w.b1, w.W2, w.b2, w.gamma, w.beta)]
+
+
+def _device_ok():
+    rs = _rs()
+    assert rs.rs_get_last_device_error() == 0
+
+
+# --------------------------------------------------------------------------- select
+@pytest.mark.parametrize("L", [1, 2, 3, 197, 1098, 1569, 4100])
+@pytest.mark.parametrize("ties", [False, True])
+def test_select_bitexact(L, ties):
+    """fp32 score finalisation and top-k: bit-exact against the oracle's selection of
+    the same fp32 keys (both sides finalise in fp32, sum left to right)."""
+    rs = _rs()
+    B, P = 3, 6
+    parts = random_partials(B, L, P, seed=L + 7 * ties, ties=ties)
+    s_ref = oracle.finalize_scores_f32(parts.numpy(), B, L)
+    ks = sorted({0, min(1, L - 1), (L - 1) // 2, max(L - 2, 0), L - 1})
+    pd = parts.to(dev)
+    for k in ks:
+        scores, kept = rs.rs_select_topk(pd, B, L, k)
+        torch.cuda.synchronize()
+        assert np.array_equal(scores.cpu().numpy(), s_ref), "fp32 scores differ"
+        for b in range(B):
+            ref = oracle.select_topk(s_ref[b].astype(np.float64), k)
+            assert kept[b].cpu().numpy().tolist() == ref.tolist(), (L, k, b)
+
+
+def test_select_cls_lowest_and_empty_batch():
+    rs = _rs()
+    B, L, P = 2, 50, 1
+    parts = random_partials(B, L, P, seed=3) + 1.0
+    parts[0] = 0.0  # CLS of sample 0 has score 0
+    scores, kept = rs.rs_select_topk(parts.to(dev), B, L, 10)
+    assert kept[0, 0].item() == 0 and 0 not in kept[0, 1:].tolist()
+    e_s, e_k = rs.rs_select_topk(torch.empty(0, 1, device=dev), 0, L, 3)
+    assert e_k.numel() == 0
+
+
+# --------------------------------------------------------------------------- gather
+@pytest.mark.parametrize("C", [64, 192, 384, 768, 1024, 2048])
+def test_gather_exact(C):
+    rs = _rs()
+    g = torch.Generator().manual_seed(C)
+    B, L, k = 5, 77, 31
+    y = torch.randn(B, L, C, generator=g).to(torch.bfloat16)
+    kept = torch.stack([torch.cat([torch.zeros(1, dtype=torch.long),
+                                   torch.sort(torch.randperm(L - 1, generator=g)[:k] + 1).values])
+                        for _ in range(B)]).to(torch.int32)
+    out = rs.rs_gather_rows(y.to(dev), kept.to(dev), k)
+    ref = np.stack([oracle.gather(y[b].float().numpy(), kept[b].numpy()) for b in range(B)])
+    assert np.array_equal(out.float().cpu().numpy(), ref)
+
+
+# --------------------------------------------------------------------------- LN stats
+@pytest.mark.parametrize("C", [64, 192, 384, 768, 1024, 2048])
+def test_ln_stats(C):
+    rs = _rs()
+    inp = random_block(3, 45, C, 64, seed=C, fg_rows=5)
+    x = inp.x.reshape(-1, C)
+    st = rs.rs_ln_stats(x.to(dev)).cpu().numpy()
+    x64 = parity.f64(x)
+    mu = x64.mean(1)
+    var = ((x64 - mu[:, None]) ** 2).mean(1)
+    assert np.allclose(st[:, 0], mu, rtol=0, atol=1e-5)
+    assert np.allclose(st[:, 1], 1 / np.sqrt(var + oracle.EPS), rtol=2e-5, atol=0)
+
+
+# --------------------------------------------------------------------------- fc1 / fc2
+@pytest.mark.parametrize("M,C,H", [(394, 192, 768), (130, 384, 1536), (77, 768, 3072),
+                                   (300, 1024, 4096), (1, 64, 64), (129, 128, 192)])
+def test_fc1_hidden(M, C, H):
+    """a = GELU(LN(x') W1^T + b1) stored as bf16, vs the oracle in fp64."""
+    rs = _rs()
+    inp = random_block(1, M, C, H, seed=M + C, fg_rows=M // 4)
+    x = inp.x.reshape(M, C)
+    w = inp.weights[0]
+    hid = rs.rs_ln_fc1_gelu(x.to(dev), w.W1.to(dev), w.b1.to(dev), w.gamma.to(dev), w.beta.to(dev))
+    w64 = parity.weights64(w)
+    ref = oracle.gelu(oracle.fc(oracle.layer_norm(parity.f64(x), w64["gamma"], w64["beta"]),
+                                w64["W1"], w64["b1"]))
+    parity.check_y(parity.f64(hid), ref, "hidden")
+    _device_ok()
+
+
+@pytest.mark.parametrize("M,C,H", [(394, 192, 768), (130, 384, 1536), (77, 768, 3072),
+                                   (300, 1024, 4096), (129, 128, 192), (5, 320, 64)])
+def test_fc2_residual_shift(M, C, H):
+    """y = x' + a W2^T + b2 and the per-row partial sums of (h - x')^2, for a given bf16
+    hidden activation a (drawn here; the same a feeds both sides)."""
+    rs = _rs()
+    inp = random_block(1, M, C, H, seed=M + H, fg_rows=M // 4)
+    x = inp.x.reshape(M, C)
+    w = inp.weights[0]
+    g = torch.Generator().manual_seed(M * 3 + 1)
+    a = (torch.randn(M, H, generator=g) * 0.3).to(torch.bfloat16)
+    y, parts = rs.rs_fc2_residual_shift(a.to(dev), x.to(dev), w.W2.to(dev), w.b2.to(dev))
+    w64 = parity.weights64(w)
+    x64 = parity.f64(x)
+    h = oracle.fc(parity.f64(a), w64["W2"], w64["b2"])
+    parity.check_y(parity.f64(y), h + x64, "y")
+    s_ref = oracle.shift_score(h, x64)
+    s_gpu = np.sqrt(parts.double().cpu().numpy().sum(1))
+    parity.check_scores(s_gpu, s_ref)
+    _device_ok()
+
+
+# --------------------------------------------------------------------------- whole block
+def _run_block(x, w, k):
+    rs = _rs()
+    W = _to_dev(w)
+    out = rs.rs_block_forward(x.to(dev), *W, k)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny_deit_t", "deit_s", "deit_b"])
+def test_block_config(name):
+    """Full batch on the GPU (the launch bench.py times); every sample of the tiny
+    config and a seeded subset of the others checked against the oracle."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, seed=0)
+    k = wl.keep_k[0]
+    gpu = _run_block(inp.x, inp.weights[0], k)
+    if name == "tiny_deit_t":
+        samples = list(range(wl.B))
+    else:
+        rng = np.random.default_rng(1)
+        samples = sorted({0, wl.B - 1, *rng.choice(wl.B, 14, replace=False).tolist()})
+    ref = parity.oracle_block(inp.x[samples], inp.weights[0], k)
+    res = parity.check_block(gpu, ref, k, samples)
+    print(name, res)
+    _device_ok()
+
+
+@pytest.mark.parametrize("name", ["umt_b", "umt_l"])
+def test_video_config(name):
+    """UMT-shaped configs at full batch; 4 sampled clips checked. Each UMT-L stage is
+    checked on the oracle's own (bf16-stored) previous-stage output."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, seed=0)
+    samples = [0, 5, 9, wl.B - 1]
+    x_gpu = inp.x
+    x_ref = inp.x[samples]
+    for s in range(wl.stages):
+        k = wl.keep_k[s]
+        x_in = x_gpu.clone()
+        x_in[samples] = x_ref  # checked clips start from the oracle's previous output
+        gpu = _run_block(x_in, inp.weights[s], k)
+        ref = parity.oracle_block(x_ref, inp.weights[s], k)
+        res = parity.check_block(gpu, ref, k, samples)
+        print(name, "stage", s, res)
+        x_gpu = gpu[0].cpu()
+        x_ref = torch.from_numpy(ref[0]).to(torch.bfloat16)
+    _device_ok()
+
+
+# --------------------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("B,L,C,H", [(3, 50, 128, 256), (1, 2, 64, 64), (2, 129, 192, 768),
+                                     (4, 197, 320, 640), (1, 1, 64, 128)])
+def test_block_edges(B, L, C, H):
+    """Ragged M (not a multiple of 128), tiny L, odd widths, every keep_k edge."""
+    inp = random_block(B, L, C, H, seed=B * L + C, fg_rows=L // 3)
+    for k in sorted({0, min(1, L - 1), max(L - 2, 0), L - 1}):
+        gpu = _run_block(inp.x, inp.weights[0], k)
+        ref = parity.oracle_block(inp.x, inp.weights[0], k)
+        parity.check_block(gpu, ref, k)
+
+
+def test_block_duplicate_rows_tie_rule():
+    """Duplicated patch rows give identical scores on both sides; the lower index wins."""
+    B, L, C, H = 2, 60, 192, 768
+    inp = random_block(B, L, C, H, seed=21, fg_rows=10)
+    x = inp.x.clone()
+    x[:, 40] = x[:, 7]
+    x[:, 41] = x[:, 7]
+    x[:, 12] = x[:, 3]
+    gpu = _run_block(x, inp.weights[0], 25)
+    s = gpu[2].cpu()
+    assert torch.equal(s[:, 40], s[:, 7]) and torch.equal(s[:, 41], s[:, 7])
+    ref = parity.oracle_block(x, inp.weights[0], 25)
+    parity.check_block(gpu, ref, 25)
+    for b in range(B):
+        kept = gpu[1][b].tolist()
+        if 40 in kept:
+            assert 7 in kept
+        if 41 in kept:
+            assert 40 in kept
+
+
+def test_block_zero_second_layer_closed_form():
+    """W2 = 0: h = b2 for every token, so y = x' + b2 (one bf16 rounding) and
+    s = ||b2 - x'||; a row equal to b2 scores 0."""
+    B, L, C, H = 2, 70, 256, 512
+    inp = random_block(B, L, C, H, seed=5)
+    w = inp.weights[0]
+    w.W2 = torch.zeros_like(w.W2)
+    x = inp.x.clone()
+    x[1, 9] = w.b2
+    gpu = _run_block(x, w, 30)
+    y_kept, kept, s = (t.cpu() for t in gpu)
+    x64 = parity.f64(x)
+    b2 = parity.f64(w.b2)
+    s_ref = np.sqrt(((x64 - b2) ** 2).sum(-1))
+    assert s[1, 9].item() == 0.0
+    assert np.allclose(s.double().numpy(), s_ref, rtol=1e-5, atol=1e-6)
+    for b in range(B):
+        rows = kept[b].long()
+        exp = torch.from_numpy(x64[b][rows.numpy()] + b2).to(torch.bfloat16)
+        assert torch.equal(y_kept[b], exp)
+
+
+def test_block_empty_batch():
+    rs = _rs()
+    inp = random_block(1, 10, 64, 64, seed=1)
+    W = _to_dev(inp.weights[0])
+    x = torch.empty(0, 10, 64, dtype=torch.bfloat16, device=dev)
+    y_kept, kept, s = rs.rs_block_forward(x, *W, 3)
+    assert y_kept.shape == (0, 4, 64)
