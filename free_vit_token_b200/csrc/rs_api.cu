@@ -96,18 +96,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major bf16 [rows, inner] viewed as tiles of {64 elements, box_rows rows},
-// 128-byte swizzled in shared memory; rows past the end read as zero.
-int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+// Row-major bf16 [rows, inner] viewed as tiles of {box_inner elements, box_rows
+// rows}: 64-wide boxes use the 128-byte swizzle (GEMM operands), 32-wide boxes
+// the 64-byte swizzle (epilogue output boxes). Rows past the end read as zero
+// and are not written.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
+              uint32_t box_inner = 64) {
   auto fn = encode_fn();
   if (fn == nullptr) return RS_ERR_CUDA;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RS_OK : RS_ERR_CUDA;
 }
 
@@ -144,9 +149,10 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
             const void* gamma, const void* beta, float* stats, void* hidden, cudaStream_t s) {
   RS_CUDA(rs::launch_ln_stats(x, M, C, stats, s));
   const int bn = rs::fc1_block_n(H);
-  CUtensorMap tmX, tmW;
+  CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, W1, C, H, bn));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
@@ -160,7 +166,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
-  RS_CUDA(rs::launch_fc1(tmX, tmW, p, bn, st.num_sms, s));
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, st.num_sms, s));
   return RS_OK;
 }
 

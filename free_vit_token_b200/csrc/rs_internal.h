@@ -32,12 +32,12 @@ struct MlpParams {
   unsigned long long timeout_ns;  // limit of one pipeline wait
 };
 
-size_t mlp_smem_bytes(int bn, bool ln, int K);
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K);
 int fc1_block_n(int H);
 int fc2_block_n(int C);
 cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, cudaStream_t stream);
-cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const MlpParams& p, int bn,
-                       int num_sms, cudaStream_t s);
+cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
+                       const MlpParams& p, int bn, int num_sms, cudaStream_t s);
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p,
                        int bn, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,

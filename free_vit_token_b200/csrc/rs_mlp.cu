@@ -33,20 +33,27 @@ constexpr int kLnWarp0 = 12;
 constexpr int kNumLnWarps = 4;
 constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 constexpr int kCtrlBytes = 512;                 // barriers, TMEM slot, abort flag
+constexpr int kEpiBoxBytes = 32 * 32 * 2;       // one warp's 32 x 32 bf16 output box
 constexpr uint32_t kTmemCols = 512;
 
 __host__ __device__ constexpr int stage_bytes(int bn) { return kAStageBytes + bn * kBK * 2; }
-__host__ __device__ constexpr int num_stages(int bn, bool ln) {
-  // LN mode keeps gamma and beta (RS_MAX_C floats each) in shared memory too.
-  return ((kSmemLimit - 1024 - kCtrlBytes - (ln ? 2 * RS_MAX_C * 4 : 0)) / stage_bytes(bn)) > 6
+__host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
+  // alignment slack + control block + gamma/beta (bf16, up to RS_MAX_C each) +
+  // the fc1 epilogue's per-warp output boxes
+  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) +
+         (epi == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0);
+}
+__host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
+  return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn) > 6
              ? 6
-             : ((kSmemLimit - 1024 - kCtrlBytes - (ln ? 2 * RS_MAX_C * 4 : 0)) / stage_bytes(bn));
+             : (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn);
 }
 __host__ __device__ constexpr int num_threads(bool ln) { return (ln ? 16 : 12) * 32; }
 
-size_t mlp_smem_bytes(int bn, bool ln, int K) {
-  return 1024 + static_cast<size_t>(num_stages(bn, ln)) * stage_bytes(bn) + kCtrlBytes +
-         (ln ? 2 * static_cast<size_t>(K) * 4 : 0);
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K) {
+  return 1024 + static_cast<size_t>(num_stages(bn, ln, epi)) * stage_bytes(bn) +
+         (epi == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0) + kCtrlBytes +
+         (ln ? 4 * static_cast<size_t>(K) : 0);
 }
 
 __device__ __forceinline__ float gelu_erf(float z) {
@@ -58,19 +65,22 @@ __device__ __forceinline__ float gelu_erf(float z) {
 template <int BN, bool LN_A, int EPI>
 __global__ void __launch_bounds__(num_threads(LN_A), 1)
     mlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const MlpParams p) {
+                    const __grid_constant__ CUtensorMap tmOut, const MlpParams p) {
   constexpr int kBStageBytes = BN * kBK * 2;
-  constexpr int STAGES = num_stages(BN, LN_A);
+  constexpr int STAGES = num_stages(BN, LN_A, EPI);
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN);
+  constexpr int kOutBytes = EPI == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(2 * BN <= static_cast<int>(kTmemCols), "TMEM double buffer");
+  static_assert(STAGES >= 2, "pipeline depth");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kAStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * kBStageBytes);
+  uint8_t* sOut = sB + STAGES * kBStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kOutBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* aready = empty + STAGES;
   uint64_t* tfull = aready + STAGES;
@@ -78,8 +88,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_gamma = reinterpret_cast<float*>(sB + STAGES * kBStageBytes + kCtrlBytes);
-  float* s_beta = s_gamma + p.K;
+  __nv_bfloat16* s_gamma = reinterpret_cast<__nv_bfloat16*>(sOut + kOutBytes + kCtrlBytes);
+  __nv_bfloat16* s_beta = s_gamma + p.K;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -102,15 +112,18 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI == kEpiGelu) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   if constexpr (LN_A) {
-    for (int i = threadIdx.x; i < p.K; i += blockDim.x) {
-      s_gamma[i] = __bfloat162float(p.ln_gamma[i]);
-      s_beta[i] = __bfloat162float(p.ln_beta[i]);
+    const uint4* g = reinterpret_cast<const uint4*>(p.ln_gamma);
+    const uint4* b = reinterpret_cast<const uint4*>(p.ln_beta);
+    for (int i = threadIdx.x; i < p.K / 8; i += blockDim.x) {
+      reinterpret_cast<uint4*>(s_gamma)[i] = __ldg(g + i);
+      reinterpret_cast<uint4*>(s_beta)[i] = __ldg(b + i);
     }
   }
   tc_fence_before_sync();
@@ -187,9 +200,16 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
     __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                          // TMEM lane quadrant of this warp
-    const int half = (warp - kEpiWarp0) >> 2;        // which half of the BN columns
+    // Warp -> TMEM lane quadrant q (rows 32q..32q+31 of the tile) and one half
+    // of the BN columns; 32-column chunks, the TMEM load of chunk n+1 in flight
+    // while chunk n is processed. The accumulator is handed back to the MMA
+    // warp as soon as its last chunk is in registers.
+    const int q = warp & 3;
+    const int half = (warp - kEpiWarp0) >> 2;
     constexpr int kHalf = BN / 2;
+    constexpr int NCH = kHalf / 32;
+    uint8_t* box = sOut + (warp - kEpiWarp0) * kEpiBoxBytes;
+    const uint32_t box_u32 = smem_u32(box);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -206,10 +226,22 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
                              static_cast<uint32_t>(acc * BN + half * kHalf);
       const int col0 = n_blk * BN + half * kHalf;
       float part = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kHalf; c += 32) {
-        uint32_t r[32];
-        tmem_load_32cols(t_row + c, r);
+      uint32_t ra[32], rb[32];
+      tmem_ld32_async(t_row, ra);
+#pragma unroll
+      for (int n = 0; n < NCH; ++n) {
+        uint32_t(&r)[32] = (n & 1) ? rb : ra;
+        uint32_t(&nx)[32] = (n & 1) ? ra : rb;
+        tmem_wait_ld();
+        reg_fence(r);
+        if (n + 1 < NCH) {
+          tmem_ld32_async(t_row + (n + 1) * 32, nx);
+        } else {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        const int c = n * 32;
         const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
         uint4 bv[4];
 #pragma unroll
@@ -222,6 +254,20 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
             const float z0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
             const float z1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
             outw[e] = pack_bf16x2(gelu_erf(z0), gelu_erf(z1));
+          }
+          // Row `lane` of this warp's 32 x 32 output box, 64-byte swizzled
+          // (16-byte chunk j of row r at j ^ ((r >> 1) & 3)), then one TMA store.
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            sts128(box_u32 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
+                   make_uint4(outw[4 * j], outw[4 * j + 1], outw[4 * j + 2], outw[4 * j + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, box, col0 + c, m_blk * kBM + q * 32);
+            bulk_commit_group();
           }
         } else {
           uint4 xv[4] = {};
@@ -242,41 +288,49 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
             part = fmaf(d0, d0, part);
             part = fmaf(d1, d1, part);
           }
-        }
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.N + col0 + c);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + off);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
+          }
         }
       }
       if constexpr (EPI == kEpiResidShift) {
         if (row_ok) p.partials[static_cast<size_t>(row) * p.num_partials + n_blk * 2 + half] = part;
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if constexpr (EPI == kEpiGelu) {
+      if (lane == 0) bulk_wait_group0();
+      __syncwarp();
     }
   } else if (LN_A && warp >= kLnWarp0) {
     // ------------------------------------------------------------ LayerNorm staging
-    // Warp j owns rows 32j .. 32j+31 of every A stage. Per pass i (0..7) the warp
-    // covers 4 rows x 128 B: lane -> row 32j + 4i + lane/8, physical 16-byte chunk
-    // lane%8, which holds logical chunk (lane%8) ^ (row%8) under the swizzle.
+    // The A stage holds raw x' (TMA, 128-byte swizzle: 16-byte chunk c of row r
+    // at physical chunk c ^ (r % 8)). Warp j normalises rows 32j .. 32j+31 in
+    // place. Lane l always handles logical chunk c = l % 8 (columns 8c .. 8c+7 of
+    // the k-block) of rows 32j + 4i + l/8, i = 0..7, so its gamma/beta slice is
+    // read once per stage and every shared access is conflict-free.
     const int j = warp - kLnWarp0;
+    const int c = lane & 7;
+    const int rsub = lane >> 3;
+    const uint32_t sA_u32 = smem_u32(sA);
+    const uint32_t g_u32 = smem_u32(s_gamma) + c * 16;
+    const uint32_t b_u32 = smem_u32(s_beta) + c * 16;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile / p.n_blocks;
-      float rstd[8], nmr[8];
+      uint64_t rs2[8], nm2[8];  // (rstd, rstd) and (-mean*rstd, -mean*rstd) per row
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int row = m_blk * kBM + 32 * j + 4 * i + (lane >> 3);
+        const int row = m_blk * kBM + 32 * j + 4 * i + rsub;
         float2 st = make_float2(0.f, 0.f);
         if (row < p.M) st = p.stats[row];
-        rstd[i] = st.y;
-        nmr[i] = -st.x * st.y;
+        rs2[i] = f2pack(st.y, st.y);
+        nm2[i] = f2pack(-st.x * st.y, -st.x * st.y);
       }
       for (int kb = 0; kb < KB; ++kb) {
         int w_ok = 1;
@@ -284,28 +338,36 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
         if (!w_ok) { ok = false; break; }
         mbar_try_wait(&full[stage], phase);  // completed: acquire for every lane
-        uint8_t* a = sA + stage * kAStageBytes;
+        const uint4 gq = lds128(g_u32 + kb * 128);
+        const uint4 bq = lds128(b_u32 + kb * 128);
+        const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+        const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+        uint64_t g2[4], b2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          g2[e] = f2pack(bf16lo(gw[e]), bf16hi(gw[e]));
+          b2[e] = f2pack(bf16lo(bw[e]), bf16hi(bw[e]));
+        }
+        const uint32_t a_u32 = sA_u32 + stage * kAStageBytes;
+        uint32_t addr[8];
+        uint4 v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int r = 32 * j + 4 * i + (lane >> 3);
-          const int pch = lane & 7;
-          const int lch = pch ^ (r & 7);
-          uint4* ptr = reinterpret_cast<uint4*>(a + r * 128 + pch * 16);
-          const uint4 v = *ptr;
-          const float4* g4 = reinterpret_cast<const float4*>(s_gamma + kb * kBK + lch * 8);
-          const float4* b4 = reinterpret_cast<const float4*>(s_beta + kb * kBK + lch * 8);
-          const float4 g0 = g4[0], g1 = g4[1], be0 = b4[0], be1 = b4[1];
-          const float xs = rstd[i], xb = nmr[i];
-          uint4 o;
-          o.x = pack_bf16x2(fmaf(fmaf(bf16lo(v.x), xs, xb), g0.x, be0.x),
-                            fmaf(fmaf(bf16hi(v.x), xs, xb), g0.y, be0.y));
-          o.y = pack_bf16x2(fmaf(fmaf(bf16lo(v.y), xs, xb), g0.z, be0.z),
-                            fmaf(fmaf(bf16hi(v.y), xs, xb), g0.w, be0.w));
-          o.z = pack_bf16x2(fmaf(fmaf(bf16lo(v.z), xs, xb), g1.x, be1.x),
-                            fmaf(fmaf(bf16hi(v.z), xs, xb), g1.y, be1.y));
-          o.w = pack_bf16x2(fmaf(fmaf(bf16lo(v.w), xs, xb), g1.z, be1.z),
-                            fmaf(fmaf(bf16hi(v.w), xs, xb), g1.w, be1.w));
-          *ptr = o;
+          const int r = 32 * j + 4 * i + rsub;
+          addr[i] = a_u32 + r * 128 + ((c ^ (r & 7)) << 4);
+          v[i] = lds128(addr[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t xw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t x2 = f2pack(bf16lo(xw[e]), bf16hi(xw[e]));
+            const float2 u = f2unpack(ffma2(ffma2(x2, rs2[i], nm2[i]), g2[e], b2[e]));
+            o[e] = pack_bf16x2(u.x, u.y);
+          }
+          sts128(addr[i], make_uint4(o[0], o[1], o[2], o[3]));
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -366,15 +428,16 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __re
 
 // ------------------------------------------------------------------ host launchers
 template <int BN, bool LN_A, int EPI>
-static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const MlpParams& p,
-                               int num_sms, cudaStream_t stream) {
+static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                               const CUtensorMap& tmOut, const MlpParams& p, int num_sms,
+                               cudaStream_t stream) {
   auto kern = mlp_gemm_kernel<BN, LN_A, EPI>;
-  const size_t smem = mlp_smem_bytes(BN, LN_A, p.K);
+  const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  kern<<<grid, num_threads(LN_A), smem, stream>>>(tmA, tmB, p);
+  kern<<<grid, num_threads(LN_A), smem, stream>>>(tmA, tmB, tmOut, p);
   return cudaGetLastError();
 }
 
@@ -398,22 +461,22 @@ int fc2_block_n(int C) {
   return C % 256 == 0 ? 256 : (C % 192 == 0 ? 192 : (C % 128 == 0 ? 128 : 64));
 }
 
-cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const MlpParams& p, int bn,
-                       int num_sms, cudaStream_t s) {
+cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
+                       const MlpParams& p, int bn, int num_sms, cudaStream_t s) {
   switch (bn) {
-    case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, p, num_sms, s);
-    case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, p, num_sms, s);
-    default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, p, num_sms, s);
+    case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+    case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+    default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
   }
 }
 
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p, int bn,
                        int num_sms, cudaStream_t s) {
   switch (bn) {
-    case 256: return launch_gemm<256, false, kEpiResidShift>(tmHid, tmW2, p, num_sms, s);
-    case 192: return launch_gemm<192, false, kEpiResidShift>(tmHid, tmW2, p, num_sms, s);
-    case 128: return launch_gemm<128, false, kEpiResidShift>(tmHid, tmW2, p, num_sms, s);
-    default: return launch_gemm<64, false, kEpiResidShift>(tmHid, tmW2, p, num_sms, s);
+    case 256: return launch_gemm<256, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
+    case 192: return launch_gemm<192, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
+    case 128: return launch_gemm<128, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
+    default: return launch_gemm<64, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
   }
 }
 
