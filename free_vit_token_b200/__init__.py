@@ -9,8 +9,10 @@ from .rs import (  # noqa: F401
     rs_block_forward,
     rs_fc2_residual_shift,
     rs_gather_rows,
+    rs_gelu_apply,
     rs_get_last_device_error,
     rs_ln_fc1_gelu,
+    rs_ln_fc1_gelu_staged,
     rs_ln_stats,
     rs_num_partials,
     rs_release_workspace,

@@ -29,8 +29,10 @@ DevState g_dev[kMaxDevices];
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Workspace: the fc1 part (LN statistics and the folded weights) first, then
+// the block's intermediates.
 struct WsLayout {
-  size_t stats, hidden, y, partials, total;
+  size_t stats, wg, colg, colc, fc1_total, hidden, y, partials, total;
 };
 
 WsLayout ws_layout(int64_t M, int C, int H) {
@@ -38,6 +40,13 @@ WsLayout ws_layout(int64_t M, int C, int H) {
   size_t off = 0;
   w.stats = off;
   off = align_up(off + static_cast<size_t>(M) * 8, 1024);
+  w.wg = off;
+  off = align_up(off + static_cast<size_t>(H) * C * 2, 1024);
+  w.colg = off;
+  off = align_up(off + static_cast<size_t>(H) * 4, 1024);
+  w.colc = off;
+  off = align_up(off + static_cast<size_t>(H) * 4, 1024);
+  w.fc1_total = off;
   w.hidden = off;
   off = align_up(off + static_cast<size_t>(M) * H * 2, 1024);
   w.y = off;
@@ -145,28 +154,44 @@ int check_rows(int64_t M, int C, int H) {
     }                                                       \
   } while (0)
 
+// LN statistics, then fc1 with the LayerNorm folded into the GEMM (default) or
+// staged into the A operand by LN warps (staged = true). `ws` holds the fc1
+// part of the workspace layout for these sizes.
 int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, const void* b1,
-            const void* gamma, const void* beta, float* stats, void* hidden, cudaStream_t s) {
-  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, s));
+            const void* gamma, const void* beta, uint8_t* ws, const WsLayout& w, void* hidden,
+            bool staged, cudaStream_t s) {
+  float* stats = reinterpret_cast<float*>(ws + w.stats);
+  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, st.num_sms, s));
   const int bn = rs::fc1_block_n(H);
-  CUtensorMap tmX, tmW, tmHid;
-  RS_TRY(make_tmap(&tmX, x, C, M, 128));
-  RS_TRY(make_tmap(&tmW, W1, C, H, bn));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
   p.K = C;
   p.n_blocks = H / bn;
   p.num_tiles = ((M + 127) / 128) * p.n_blocks;
-  p.ln_gamma = static_cast<const __nv_bfloat16*>(gamma);
-  p.ln_beta = static_cast<const __nv_bfloat16*>(beta);
   p.stats = reinterpret_cast<const float2*>(stats);
-  p.bias = static_cast<const __nv_bfloat16*>(b1);
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
-  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, st.num_sms, s));
+  const void* wB = W1;
+  if (staged) {
+    p.ln_gamma = static_cast<const __nv_bfloat16*>(gamma);
+    p.ln_beta = static_cast<const __nv_bfloat16*>(beta);
+    p.bias = static_cast<const __nv_bfloat16*>(b1);
+  } else {
+    void* wg = ws + w.wg;
+    float* colg = reinterpret_cast<float*>(ws + w.colg);
+    float* colc = reinterpret_cast<float*>(ws + w.colc);
+    RS_CUDA(rs::launch_ln_fold(W1, gamma, beta, b1, H, C, wg, colg, colc, st.num_sms, s));
+    p.colG = colg;
+    p.colC = colc;
+    wB = wg;
+  }
+  CUtensorMap tmX, tmW, tmHid;
+  RS_TRY(make_tmap(&tmX, x, C, M, 128));
+  RS_TRY(make_tmap(&tmW, wB, C, H, bn));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, st.num_sms, s));
   return RS_OK;
 }
 
@@ -224,12 +249,20 @@ int rs_ln_stats(const void* x, int M, int C, float* stats, void* stream) {
   if (M == 0) return RS_OK;
   if (!x || !stats) return RS_ERR_NULL;
   if (!al16(x) || !al8(stats)) return RS_ERR_ALIGN;
-  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, static_cast<cudaStream_t>(stream)));
+  int num_sms = 148;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevState* st = nullptr;
+    RS_TRY(dev_state(&st));
+    num_sms = st->num_sms;
+  }
+  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, num_sms, static_cast<cudaStream_t>(stream)));
   return RS_OK;
 }
 
-int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
-                   const void* gamma, const void* beta, void* hidden, void* stream) {
+static int ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                       const void* gamma, const void* beta, void* hidden, bool staged,
+                       void* stream) {
   RS_TRY(check_width(C));
   RS_TRY(check_hidden(H));
   RS_TRY(check_rows(M, C, H));
@@ -240,9 +273,29 @@ int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const voi
   std::lock_guard<std::mutex> lock(g_mu);
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
-  RS_TRY(ensure_ws(*st, align_up(static_cast<size_t>(M) * 8, 1024)));
-  return run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, static_cast<float*>(st->ws), hidden,
-                 static_cast<cudaStream_t>(stream));
+  const WsLayout w = ws_layout(M, C, H);
+  RS_TRY(ensure_ws(*st, w.fc1_total));
+  return run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, static_cast<uint8_t*>(st->ws), w, hidden,
+                 staged, static_cast<cudaStream_t>(stream));
+}
+
+int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                   const void* gamma, const void* beta, void* hidden, void* stream) {
+  return ln_fc1_gelu(x, M, C, H, W1, b1, gamma, beta, hidden, false, stream);
+}
+
+int rs_ln_fc1_gelu_staged(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                          const void* gamma, const void* beta, void* hidden, void* stream) {
+  return ln_fc1_gelu(x, M, C, H, W1, b1, gamma, beta, hidden, true, stream);
+}
+
+int rs_gelu_apply(const float* z, float* out, int n, void* stream) {
+  if (n < 0) return RS_ERR_SHAPE;
+  if (n == 0) return RS_OK;
+  if (!z || !out) return RS_ERR_NULL;
+  if (!al4(z) || !al4(out)) return RS_ERR_ALIGN;
+  RS_CUDA(rs::launch_gelu(z, out, n, static_cast<cudaStream_t>(stream)));
+  return RS_OK;
 }
 
 int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H, const void* W2,
@@ -320,13 +373,12 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
   const WsLayout w = ws_layout(M, C, H);
   RS_TRY(ensure_ws(*st, w.total));
   uint8_t* ws = static_cast<uint8_t*>(st->ws);
-  float* stats = reinterpret_cast<float*>(ws + w.stats);
   void* hidden = ws + w.hidden;
   void* y = ws + w.y;
   float* partials = reinterpret_cast<float*>(ws + w.partials);
   const int np = 2 * C / rs::fc2_block_n(C);
 
-  RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, stats, hidden, s));
+  RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
   RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s));
   RS_CUDA(rs::launch_select(partials, np, B, L, keep_k, scores, kept_idx, s));
   RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k, y_kept, st->num_sms, s));

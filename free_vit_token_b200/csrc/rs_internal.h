@@ -15,6 +15,7 @@ namespace rs {
 constexpr float kLnEps = 1e-6f;          // LayerNorm epsilon (the pages do not state one)
 constexpr int kEpiGelu = 0;              // fc1 epilogue: + b1, erf-GELU, bf16 store
 constexpr int kEpiResidShift = 1;        // fc2 epilogue: + b2, residual, shift partials
+constexpr int kEpiGeluFold = 2;          // fc1 epilogue: folded LN (mean, rstd, G, cb), erf-GELU
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // one pipeline wait: 4 s
 
 struct MlpParams {
@@ -23,6 +24,8 @@ struct MlpParams {
   const __nv_bfloat16* ln_gamma;  // [K]   fc1 only
   const __nv_bfloat16* ln_beta;   // [K]   fc1 only
   const float2* stats;            // [M]   fc1 only: (mean, rstd) per row
+  const float* colG;              // [N]   folded-LN fc1: sum_c Wg[j, c]
+  const float* colC;              // [N]   folded-LN fc1: sum_c W1[j, c] beta[c] + b1[j]
   const __nv_bfloat16* bias;      // [N]
   __nv_bfloat16* out;             // [M, N] hidden (fc1) or y (fc2)
   const __nv_bfloat16* resid;     // [M, N] x' (fc2 only)
@@ -35,9 +38,14 @@ struct MlpParams {
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K);
 int fc1_block_n(int H);
 int fc2_block_n(int C);
-cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, cudaStream_t stream);
+cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
+                            cudaStream_t stream);
+cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,
+                           int H, int C, void* Wg, float* colG, float* colC, int num_sms,
+                           cudaStream_t stream);
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, int num_sms, cudaStream_t s);
+                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s);
+cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream);
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p,
                        int bn, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,

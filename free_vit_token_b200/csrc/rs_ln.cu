@@ -1,0 +1,175 @@
+// rs_ln.cu -- the LayerNorm pieces of the MLP sublayer (§3.3 Eq. (6) of
+// "Representation Shift: Unifying Token Compression with FlashAttention"):
+//
+//   ln_stats:  per row r of x', mean_r and rstd_r = 1/sqrt(var_r + eps) (biased
+//              variance), one warp per row, two passes over the row held in
+//              registers, reductions by warp shuffles.
+//   ln_fold:   the LayerNorm's affine part folded into fc1's weights. With
+//              u = (x' - mean) * rstd * gamma + beta,
+//                W1 u + b1 = rstd * (Wg x' - mean * G) + cb,
+//              Wg[j, c] = bf16(W1[j, c] * gamma[c]), G[j] = sum_c Wg[j, c],
+//              cb[j] = sum_c W1[j, c] * beta[c] + b1[j]. G is summed from the
+//              rounded Wg so that the mean cancels exactly in exact arithmetic.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rs_internal.h"
+#include "rs_ptx.cuh"
+
+namespace rs {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int VPL>
+__device__ __forceinline__ void load_row(const uint4* __restrict__ xr, int lane, int nvec,
+                                         uint4 (&v)[VPL]) {
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int idx = lane + 32 * i;
+    v[i] = idx < nvec ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Persistent: each warp walks rows with a grid-wide stride and keeps the next
+// row's loads in flight while it reduces the current one.
+template <int VPL>
+__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int M,
+                                                       int C, float2* __restrict__ stats) {
+  const int lane = threadIdx.x & 31;
+  const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nvec = C >> 3;
+  const float inv_c = 1.0f / static_cast<float>(C);
+  uint4 cur[VPL], nxt[VPL];
+  if (row < M) load_row<VPL>(reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * C), lane,
+                             nvec, cur);
+  for (; row < M; row += nw) {
+    const int nrow = row + nw;
+    if (nrow < M)
+      load_row<VPL>(reinterpret_cast<const uint4*>(x + static_cast<size_t>(nrow) * C), lane, nvec,
+                    nxt);
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&cur[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sum += bf16lo(w[e]) + bf16hi(w[e]);
+    }
+    const float mean = warp_sum(sum) * inv_c;
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      if (lane + 32 * i < nvec) {
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&cur[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float d0 = bf16lo(w[e]) - mean, d1 = bf16hi(w[e]) - mean;
+          sq = fmaf(d0, d0, sq);
+          sq = fmaf(d1, d1, sq);
+        }
+      }
+    }
+    sq = warp_sum(sq);
+    if (lane == 0) stats[row] = make_float2(mean, rsqrtf(sq * inv_c + kLnEps));
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) cur[i] = nxt[i];
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256)
+    ln_fold_kernel(const __nv_bfloat16* __restrict__ W1, const __nv_bfloat16* __restrict__ gamma,
+                   const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ b1,
+                   int H, int C, __nv_bfloat16* __restrict__ Wg, float* __restrict__ colG,
+                   float* __restrict__ colC) {
+  const int lane = threadIdx.x & 31;
+  const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  const int nvec = C >> 3;
+  const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
+  const uint4* b4 = reinterpret_cast<const uint4*>(beta);
+  uint4 gv[VPL], bv[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int idx = lane + 32 * i;
+    gv[i] = idx < nvec ? __ldg(g4 + idx) : make_uint4(0, 0, 0, 0);
+    bv[i] = idx < nvec ? __ldg(b4 + idx) : make_uint4(0, 0, 0, 0);
+  }
+  for (int j = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); j < H; j += nw) {
+    const uint4* wr = reinterpret_cast<const uint4*>(W1 + static_cast<size_t>(j) * C);
+    uint4* out = reinterpret_cast<uint4*>(Wg + static_cast<size_t>(j) * C);
+    float gs = 0.f, cs = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < nvec) {
+        const uint4 wv = __ldg(wr + idx);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&wv);
+        const uint32_t* g = reinterpret_cast<const uint32_t*>(&gv[i]);
+        const uint32_t* b = reinterpret_cast<const uint32_t*>(&bv[i]);
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float w0 = bf16lo(w[e]), w1 = bf16hi(w[e]);
+          o[e] = pack_bf16x2(w0 * bf16lo(g[e]), w1 * bf16hi(g[e]));
+          gs += bf16lo(o[e]) + bf16hi(o[e]);
+          cs = fmaf(w0, bf16lo(b[e]), cs);
+          cs = fmaf(w1, bf16hi(b[e]), cs);
+        }
+        out[idx] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    gs = warp_sum(gs);
+    cs = warp_sum(cs);
+    if (lane == 0) {
+      colG[j] = gs;
+      colC[j] = cs + __bfloat162float(b1[j]);
+    }
+  }
+}
+
+cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
+                            cudaStream_t stream) {
+  const int warps = (M + 1) / 2;  // two rows per warp on average keeps loads in flight
+  int blocks = (warps + 7) / 8;
+  if (blocks > num_sms * 8) blocks = num_sms * 8;
+  if (blocks < 1) blocks = 1;
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  auto* sp = reinterpret_cast<float2*>(stats);
+  if (C <= 256)
+    ln_stats_kernel<1><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
+  else if (C <= 512)
+    ln_stats_kernel<2><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
+  else if (C <= 1024)
+    ln_stats_kernel<4><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
+  else
+    ln_stats_kernel<8><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,
+                           int H, int C, void* Wg, float* colG, float* colC, int num_sms,
+                           cudaStream_t stream) {
+  int blocks = (H + 7) / 8;
+  if (blocks > num_sms * 4) blocks = num_sms * 4;
+  const auto* w = static_cast<const __nv_bfloat16*>(W1);
+  const auto* g = static_cast<const __nv_bfloat16*>(gamma);
+  const auto* b = static_cast<const __nv_bfloat16*>(beta);
+  const auto* bb = static_cast<const __nv_bfloat16*>(b1);
+  auto* o = static_cast<__nv_bfloat16*>(Wg);
+  if (C <= 256)
+    ln_fold_kernel<1><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
+  else if (C <= 512)
+    ln_fold_kernel<2><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
+  else if (C <= 1024)
+    ln_fold_kernel<4><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
+  else
+    ln_fold_kernel<8><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
+  return cudaGetLastError();
+}
+
+}  // namespace rs

@@ -1,18 +1,21 @@
 // rs_mlp.cu -- the two contractions of the MLP sublayer (§3.3 Eq. (6) of
 // "Representation Shift: Unifying Token Compression with FlashAttention") as
-// persistent, warp-specialised tcgen05 GEMMs for sm_100a, plus the LayerNorm
-// row-statistics pass that feeds fc1's operand staging.
+// persistent, warp-specialised tcgen05 GEMMs for sm_100a.
 //
-//   fc1:  a = GELU(LN(x') W1^T + b1)           A = x' tiles (TMA), normalised
-//                                              in shared memory by LN warps
+//   fc1 (folded LN, default):  z = rstd * (x' Wg^T - mean * G) + cb, a = GELU(z)
+//        A = raw x' tiles (TMA); the LayerNorm is applied in the epilogue
+//        through the fold of rs_ln.cu (Wg = W1 * gamma).
+//   fc1 (staged LN):           a = GELU(LN(x') W1^T + b1); A = x' tiles (TMA)
+//        normalised in place in shared memory by LN warps before the MMA.
 //   fc2:  h = a W2^T + b2; y = x' + h;          A = a tiles (TMA)
 //         P[r, j] = sum_{c in group j} (h - x')^2   -- Eq. (4) with D = L2
 //
 // One CTA per SM loops over 128 x BN output tiles. Warp roles:
 //   warp 0      TMA producer (A and B tiles, 64-wide K blocks, STAGES deep ring)
 //   warp 1      TMEM owner and UMMA issuer (tcgen05.mma, M=128, N=BN, K=16)
-//   warps 4-11  epilogue: TMEM -> registers -> bias/GELU or residual/shift -> HBM
-//   warps 12-15 (fc1 only) LayerNorm staging of the A tile in place
+//   warps 4-11  epilogue: TMEM -> registers -> LN fold / bias, GELU or
+//               residual/shift -> HBM (fc1 through per-warp TMA-store boxes)
+//   warps 12-15 (staged-LN fc1 only) LayerNorm staging of the A tile in place
 // The fp32 accumulator is double-buffered in TMEM (2 x BN columns) so the
 // epilogue of one tile overlaps the main loop of the next.
 #include <cstdint>
@@ -20,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include "rs_internal.h"
+#include "rs_gelu_poly.h"
 #include "rs_ptx.cuh"
 
 namespace rs {
@@ -41,7 +45,7 @@ __host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
   // alignment slack + control block + gamma/beta (bf16, up to RS_MAX_C each) +
   // the fc1 epilogue's per-warp output boxes
   return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) +
-         (epi == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0);
+         (epi != kEpiResidShift ? kNumEpiWarps * kEpiBoxBytes : 0);
 }
 __host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
   return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn) > 6
@@ -52,14 +56,59 @@ __host__ __device__ constexpr int num_threads(bool ln) { return (ln ? 16 : 12) *
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K) {
   return 1024 + static_cast<size_t>(num_stages(bn, ln, epi)) * stage_bytes(bn) +
-         (epi == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0) + kCtrlBytes +
+         (epi != kEpiResidShift ? kNumEpiWarps * kEpiBoxBytes : 0) + kCtrlBytes +
          (ln ? 4 * static_cast<size_t>(K) : 0);
 }
 
-__device__ __forceinline__ float gelu_erf(float z) {
-  // exact GELU: z * Phi(z) = z/2 * (1 + erf(z / sqrt 2))
-  const float hz = 0.5f * z;
-  return fmaf(hz, erff(z * 0.70710678118654752f), hz);
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t kpair(float c) { return f2pack(c, c); }
+
+// Exact (erf) GELU of two fp32 lanes, GELU(z) = z * Phi(z), evaluated with the
+// polynomial of rs_gelu_poly.h (max |error| 1.1e-6, max |Phi error| 2.5e-7 in
+// float32) using paired fp32 FMAs:
+//   u = min(K z^2 - 1, 1), Phi = sat(1/2 + z P(u)).
+__device__ __forceinline__ uint64_t gelu2(uint64_t z2) {
+  uint64_t u2 = ffma2(fmul2(z2, kpair(RS_GELU_K)), z2, kpair(-1.f));
+  const float2 uf = f2unpack(u2);
+  u2 = f2pack(fminf(uf.x, 1.f), fminf(uf.y, 1.f));
+  uint64_t p = kpair(RS_GELU_P13);
+  p = ffma2(p, u2, kpair(RS_GELU_P12));
+  p = ffma2(p, u2, kpair(RS_GELU_P11));
+  p = ffma2(p, u2, kpair(RS_GELU_P10));
+  p = ffma2(p, u2, kpair(RS_GELU_P9));
+  p = ffma2(p, u2, kpair(RS_GELU_P8));
+  p = ffma2(p, u2, kpair(RS_GELU_P7));
+  p = ffma2(p, u2, kpair(RS_GELU_P6));
+  p = ffma2(p, u2, kpair(RS_GELU_P5));
+  p = ffma2(p, u2, kpair(RS_GELU_P4));
+  p = ffma2(p, u2, kpair(RS_GELU_P3));
+  p = ffma2(p, u2, kpair(RS_GELU_P2));
+  p = ffma2(p, u2, kpair(RS_GELU_P1));
+  p = ffma2(p, u2, kpair(RS_GELU_P0));
+  const float2 zf = f2unpack(z2), pf = f2unpack(p);
+  return fmul2(z2, f2pack(__saturatef(fmaf(zf.x, pf.x, 0.5f)), __saturatef(fmaf(zf.y, pf.y, 0.5f))));
+}
+
+// Elementwise GELU with the same arithmetic as the fc1 epilogue.
+__global__ void gelu_apply_kernel(const float* __restrict__ z, float* __restrict__ out, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 g = f2unpack(gelu2(f2pack(z[i], z[i + 1])));
+    out[i] = g.x;
+    out[i + 1] = g.y;
+  } else if (i < n) {
+    out[i] = f2unpack(gelu2(f2pack(z[i], 0.f))).x;
+  }
+}
+
+cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  gelu_apply_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(z, out, n);
+  return cudaGetLastError();
 }
 
 template <int BN, bool LN_A, int EPI>
@@ -69,7 +118,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   constexpr int kBStageBytes = BN * kBK * 2;
   constexpr int STAGES = num_stages(BN, LN_A, EPI);
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN);
-  constexpr int kOutBytes = EPI == kEpiGelu ? kNumEpiWarps * kEpiBoxBytes : 0;
+  constexpr bool kGeluOut = EPI != kEpiResidShift;  // fc1: GELU, TMA-store boxes
+  constexpr int kOutBytes = kGeluOut ? kNumEpiWarps * kEpiBoxBytes : 0;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(2 * BN <= static_cast<int>(kTmemCols), "TMEM double buffer");
   static_assert(STAGES >= 2, "pipeline depth");
@@ -112,7 +162,7 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI == kEpiGelu) tma_prefetch_desc(&tmOut);
+    if (kGeluOut) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -226,6 +276,13 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
                              static_cast<uint32_t>(acc * BN + half * kHalf);
       const int col0 = n_blk * BN + half * kHalf;
       float part = 0.f;
+      uint64_t nmu2 = 0, rs2 = 0;  // folded LN: (-mean, -mean), (rstd, rstd) of this row
+      if constexpr (EPI == kEpiGeluFold) {
+        float2 st = make_float2(0.f, 0.f);
+        if (row_ok) st = p.stats[row];
+        nmu2 = f2pack(-st.x, -st.x);
+        rs2 = f2pack(st.y, st.y);
+      }
       uint32_t ra[32], rb[32];
       tmem_ld32_async(t_row, ra);
 #pragma unroll
@@ -242,18 +299,37 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
         const int c = n * 32;
-        const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
-        uint4 bv[4];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) bv[v] = __ldg(bptr + v);
-        const uint32_t* bw = reinterpret_cast<const uint32_t*>(bv);
         uint32_t outw[16];
-        if constexpr (EPI == kEpiGelu) {
+        if constexpr (kGeluOut) {
+          if constexpr (EPI == kEpiGeluFold) {
+            // z = rstd * (acc - mean * G[col]) + cb[col], two columns per step
+            const ulonglong2* gp = reinterpret_cast<const ulonglong2*>(p.colG + col0 + c);
+            const ulonglong2* cp = reinterpret_cast<const ulonglong2*>(p.colC + col0 + c);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float z0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-            const float z1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-            outw[e] = pack_bf16x2(gelu_erf(z0), gelu_erf(z1));
+            for (int v = 0; v < 8; ++v) {
+              const ulonglong2 g4 = __ldg(gp + v), c4 = __ldg(cp + v);
+              const uint64_t za = ffma2(rs2, ffma2(nmu2, g4.x, f2pack(__uint_as_float(r[4 * v]),
+                                                                      __uint_as_float(r[4 * v + 1]))),
+                                        c4.x);
+              const uint64_t zb = ffma2(rs2, ffma2(nmu2, g4.y, f2pack(__uint_as_float(r[4 * v + 2]),
+                                                                      __uint_as_float(r[4 * v + 3]))),
+                                        c4.y);
+              const float2 ga = f2unpack(gelu2(za)), gb = f2unpack(gelu2(zb));
+              outw[2 * v] = pack_bf16x2(ga.x, ga.y);
+              outw[2 * v + 1] = pack_bf16x2(gb.x, gb.y);
+            }
+          } else {
+            const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
+            uint4 bv[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) bv[v] = __ldg(bptr + v);
+            const uint32_t* bw = reinterpret_cast<const uint32_t*>(bv);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 g = f2unpack(gelu2(f2pack(__uint_as_float(r[2 * e]) + bf16lo(bw[e]),
+                                                     __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]))));
+              outw[e] = pack_bf16x2(g.x, g.y);
+            }
           }
           // Row `lane` of this warp's 32 x 32 output box, 64-byte swizzled
           // (16-byte chunk j of row r at j ^ ((r >> 1) & 3)), then one TMA store.
@@ -270,6 +346,11 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
             bulk_commit_group();
           }
         } else {
+          const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
+          uint4 bv[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) bv[v] = __ldg(bptr + v);
+          const uint32_t* bw = reinterpret_cast<const uint32_t*>(bv);
           uint4 xv[4] = {};
           const size_t off = static_cast<size_t>(row) * p.N + col0 + c;
           if (row_ok) {
@@ -301,7 +382,7 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    if constexpr (EPI == kEpiGelu) {
+    if constexpr (kGeluOut) {
       if (lane == 0) bulk_wait_group0();
       __syncwarp();
     }
@@ -384,48 +465,6 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   }
 }
 
-// ------------------------------------------------------------------ LN statistics
-// One warp per row: mean and 1/sqrt(biased var + eps), two passes over the row
-// held in registers, reductions by warp shuffles.
-template <int VPL>
-__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int M,
-                                                       int C, float2* __restrict__ stats) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= M) return;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * C);
-  const int nvec = C >> 3;
-  uint4 v[VPL];
-  float sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int idx = lane + 32 * i;
-    v[i] = idx < nvec ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sum += bf16lo(w[e]) + bf16hi(w[e]);
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float mean = sum / static_cast<float>(C);
-  float sq = 0.f;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    if (lane + 32 * i < nvec) {
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float d0 = bf16lo(w[e]) - mean, d1 = bf16hi(w[e]) - mean;
-        sq = fmaf(d0, d0, sq);
-        sq = fmaf(d1, d1, sq);
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  if (lane == 0) stats[row] = make_float2(mean, rsqrtf(sq / static_cast<float>(C) + kLnEps));
-}
-
 // ------------------------------------------------------------------ host launchers
 template <int BN, bool LN_A, int EPI>
 static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
@@ -441,32 +480,24 @@ static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
   return cudaGetLastError();
 }
 
-cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, cudaStream_t stream) {
-  const int grid = (M + 7) / 8;
-  const auto* xp = static_cast<const __nv_bfloat16*>(x);
-  auto* sp = reinterpret_cast<float2*>(stats);
-  if (C <= 256)
-    ln_stats_kernel<1><<<grid, 256, 0, stream>>>(xp, M, C, sp);
-  else if (C <= 512)
-    ln_stats_kernel<2><<<grid, 256, 0, stream>>>(xp, M, C, sp);
-  else if (C <= 1024)
-    ln_stats_kernel<4><<<grid, 256, 0, stream>>>(xp, M, C, sp);
-  else
-    ln_stats_kernel<8><<<grid, 256, 0, stream>>>(xp, M, C, sp);
-  return cudaGetLastError();
-}
-
 int fc1_block_n(int H) { return H % 256 == 0 ? 256 : (H % 128 == 0 ? 128 : 64); }
 int fc2_block_n(int C) {
   return C % 256 == 0 ? 256 : (C % 192 == 0 ? 192 : (C % 128 == 0 ? 128 : 64));
 }
 
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, int num_sms, cudaStream_t s) {
+                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s) {
+  if (staged_ln) {
+    switch (bn) {
+      case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+      case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+      default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+    }
+  }
   switch (bn) {
-    case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
-    case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
-    default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+    case 256: return launch_gemm<256, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
+    case 128: return launch_gemm<128, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
+    default: return launch_gemm<64, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
   }
 }
 

@@ -30,6 +30,8 @@ SIGNATURES = {
                               _fp, _vp]),
     "rs_ln_stats": (_i, [_vp, _i, _i, _fp, _vp]),
     "rs_ln_fc1_gelu": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "rs_ln_fc1_gelu_staged": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "rs_gelu_apply": (_i, [_fp, _fp, _i, _vp]),
     "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_num_partials": (_i, [_i]),
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
@@ -129,6 +131,25 @@ def rs_ln_fc1_gelu(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: Optional[torc
                               _ptr(hidden), _stream(stream))
     _check(st, "rs_ln_fc1_gelu")
     return hidden
+
+
+def rs_ln_fc1_gelu_staged(x2d: torch.Tensor, W1, b1, gamma, beta,
+                          hidden: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, C = x2d.shape
+    H = W1.shape[0]
+    if hidden is None:
+        hidden = torch.empty(M, H, dtype=torch.bfloat16, device=x2d.device)
+    st = lib().rs_ln_fc1_gelu_staged(_ptr(x2d), M, C, H, _ptr(W1), _ptr(b1), _ptr(gamma),
+                                     _ptr(beta), _ptr(hidden), _stream(stream))
+    _check(st, "rs_ln_fc1_gelu_staged")
+    return hidden
+
+
+def rs_gelu_apply(z: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty_like(z)
+    _check(lib().rs_gelu_apply(_ptr(z), _ptr(out), z.numel(), _stream(stream)), "rs_gelu_apply")
+    return out
 
 
 def rs_num_partials(C: int) -> int:

@@ -94,11 +94,25 @@ int rs_block_forward(const void* x, int B, int L, int C, int H,
  * x [M, C] bf16; stats [M, 2] fp32 (8-byte aligned). */
 int rs_ln_stats(const void* x, int M, int C, float* stats, void* stream);
 
-/* a = GELU(LN(x') W1^T + b1) as bf16 [M, H], the LN applied while staging
- * fc1's A operand (uses rs_ln_stats internally; its stats live in the
- * library workspace). x [M, C]; hidden [M, H] bf16 output. */
+/* a = GELU(LN(x') W1^T + b1) as bf16 [M, H] (Eq. (6)'s LN and fc1 with the
+ * exact GELU). LN is fused into fc1 by folding: with Wg = bf16(W1 * gamma),
+ * G[j] = sum_c Wg[j, c] and cb[j] = sum_c W1[j, c] beta[c] + b1[j],
+ *   LN(x') W1^T + b1 = rstd * (x' Wg^T - mean * G) + cb,
+ * so the GEMM reads x' as stored and the epilogue applies mean, rstd, G, cb.
+ * Uses rs_ln_stats internally; the statistics and the folded weights live in
+ * the library workspace. x [M, C]; hidden [M, H] bf16 output. */
 int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
                    const void* gamma, const void* beta, void* hidden, void* stream);
+
+/* The same result with the LayerNorm applied while staging fc1's A operand:
+ * LN warps normalise each x' tile in shared memory (fp32 math, bf16 out)
+ * before the tensor cores read it. Same arguments and workspace use. */
+int rs_ln_fc1_gelu_staged(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                          const void* gamma, const void* beta, void* hidden, void* stream);
+
+/* The exact GELU, z * Phi(z), elementwise in fp32 with the arithmetic of the
+ * fc1 epilogue (|error| <= 1.2e-6). z, out: [n] fp32 (4-byte aligned). */
+int rs_gelu_apply(const float* z, float* out, int n, void* stream);
 
 /* fc2 with the residual and the shift partials (Eq. (6) and Eq. (4)):
  *   h = hidden W2^T + b2 (fp32), y = bf16(x' + h) [M, C],

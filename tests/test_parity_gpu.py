@@ -87,21 +87,55 @@ def test_ln_stats(C):
     assert np.allclose(st[:, 1], 1 / np.sqrt(var + oracle.EPS), rtol=2e-5, atol=0)
 
 
+# --------------------------------------------------------------------------- GELU
+def test_gelu_apply_error_bound():
+    """The epilogue's GELU against the exact z * Phi(z) (fp64 oracle) on a dense grid:
+    |error| <= 1.5e-6 everywhere and <= 3e-7 * max(1, |z|) relative to scale."""
+    rs = _rs()
+    z = torch.cat([torch.linspace(-12, 12, 400001), torch.randn(100000) * 3,
+                   torch.tensor([0.0, -0.0, 1e-30, -1e-30, 5.3, -5.3, 40.0, -40.0])]).float()
+    g = rs.rs_gelu_apply(z.to(dev)).cpu().double().numpy()
+    ref = oracle.gelu(z.double().numpy())
+    err = np.abs(g - ref)
+    assert err.max() <= 1.5e-6, err.max()
+    small = np.abs(z.numpy()) < 1e-3
+    assert np.all(err[small] <= 1e-6 * np.abs(ref[small]) + 1e-37)
+
+
 # --------------------------------------------------------------------------- fc1 / fc2
+@pytest.mark.parametrize("variant", ["folded", "staged"])
 @pytest.mark.parametrize("M,C,H", [(394, 192, 768), (130, 384, 1536), (77, 768, 3072),
                                    (300, 1024, 4096), (1, 64, 64), (129, 128, 192)])
-def test_fc1_hidden(M, C, H):
-    """a = GELU(LN(x') W1^T + b1) stored as bf16, vs the oracle in fp64."""
+def test_fc1_hidden(M, C, H, variant):
+    """a = GELU(LN(x') W1^T + b1) stored as bf16, vs the oracle in fp64: the LN folded
+    into the GEMM (default) and the LN staged into the A operand."""
     rs = _rs()
     inp = random_block(1, M, C, H, seed=M + C, fg_rows=M // 4)
     x = inp.x.reshape(M, C)
     w = inp.weights[0]
-    hid = rs.rs_ln_fc1_gelu(x.to(dev), w.W1.to(dev), w.b1.to(dev), w.gamma.to(dev), w.beta.to(dev))
+    fn = rs.rs_ln_fc1_gelu if variant == "folded" else rs.rs_ln_fc1_gelu_staged
+    hid = fn(x.to(dev), w.W1.to(dev), w.b1.to(dev), w.gamma.to(dev), w.beta.to(dev))
     w64 = parity.weights64(w)
     ref = oracle.gelu(oracle.fc(oracle.layer_norm(parity.f64(x), w64["gamma"], w64["beta"]),
                                 w64["W1"], w64["b1"]))
     parity.check_y(parity.f64(hid), ref, "hidden")
     _device_ok()
+
+
+def test_fc1_large_mean_rows():
+    """Rows with a large common offset (mean >> std): the folded LN subtracts
+    mean * G after the GEMM, so check it against the oracle on such rows."""
+    rs = _rs()
+    M, C, H = 256, 768, 1536
+    inp = random_block(1, M, C, H, seed=77)
+    x = (inp.x.float().reshape(M, C) + torch.linspace(-30, 30, M)[:, None]).to(torch.bfloat16)
+    w = inp.weights[0]
+    w64 = parity.weights64(w)
+    ref = oracle.gelu(oracle.fc(oracle.layer_norm(parity.f64(x), w64["gamma"], w64["beta"]),
+                                w64["W1"], w64["b1"]))
+    for fn in (rs.rs_ln_fc1_gelu, rs.rs_ln_fc1_gelu_staged):
+        hid = fn(x.to(dev), w.W1.to(dev), w.b1.to(dev), w.gamma.to(dev), w.beta.to(dev))
+        parity.check_y(parity.f64(hid), ref, fn.__name__)
 
 
 @pytest.mark.parametrize("M,C,H", [(394, 192, 768), (130, 384, 1536), (77, 768, 3072),
