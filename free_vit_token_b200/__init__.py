@@ -12,6 +12,7 @@ from .rs import (  # noqa: F401
     rs_gelu_apply,
     rs_get_last_device_error,
     rs_ln_fc1_gelu,
+    rs_ln_fc1_gelu_noalloc,
     rs_ln_fc1_gelu_staged,
     rs_ln_stats,
     rs_num_partials,

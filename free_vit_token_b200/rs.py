@@ -32,6 +32,7 @@ SIGNATURES = {
     "rs_ln_fc1_gelu": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_ln_fc1_gelu_staged": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_gelu_apply": (_i, [_fp, _fp, _i, _vp]),
+    "rs_ln_fc1_gelu_noalloc": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_num_partials": (_i, [_i]),
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
@@ -142,6 +143,18 @@ def rs_ln_fc1_gelu_staged(x2d: torch.Tensor, W1, b1, gamma, beta,
     st = lib().rs_ln_fc1_gelu_staged(_ptr(x2d), M, C, H, _ptr(W1), _ptr(b1), _ptr(gamma),
                                      _ptr(beta), _ptr(hidden), _stream(stream))
     _check(st, "rs_ln_fc1_gelu_staged")
+    return hidden
+
+
+def rs_ln_fc1_gelu_noalloc(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: torch.Tensor,
+                           stream=None) -> torch.Tensor:
+    """rs_ln_fc1_gelu with its scratch in the library's static device array (the caller
+    provides ``hidden``; nothing is allocated)."""
+    M, C = x2d.shape
+    H = W1.shape[0]
+    st = lib().rs_ln_fc1_gelu_noalloc(_ptr(x2d), M, C, H, _ptr(W1), _ptr(b1), _ptr(gamma),
+                                      _ptr(beta), _ptr(hidden), _stream(stream))
+    _check(st, "rs_ln_fc1_gelu_noalloc")
     return hidden
 
 

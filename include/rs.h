@@ -142,6 +142,29 @@ int rs_select_topk(const float* partials, int num_partials, int B, int L, int ke
 int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
                    void* y_kept, void* stream);
 
+/* rs_ln_fc1_gelu without any allocation, for callers that cannot allocate
+ * device memory when they call: code running while a stream is captured into
+ * a CUDA graph (where cudaMalloc is not allowed), or a host framework that
+ * hands out all device memory from its own pool. The paper has no counterpart;
+ * this is a library convenience.
+ *   Same arguments and result as rs_ln_fc1_gelu. Its scratch (LN statistics and
+ *   folded fc1 weights) is one static device array of about 8.6 MiB that every
+ *   GPU loading the library holds until exit; the call itself makes no
+ *   cudaMalloc, cudaFree or other allocating call.
+ *   Limits: M <= 65536 and H * C <= 4194304, beyond which it returns
+ *   RS_ERR_SHAPE without launching (as for any other shape error).
+ *   The first call on a device resolves the array's device address for that
+ *   device (cudaGetSymbolAddress); make that first call before any stream
+ *   capture begins.
+ *   Every call on a device shares the one array and leaves its contents behind;
+ *   each call writes every scratch byte it reads before reading it, so nothing
+ *   must start at zero. Calls whose executions overlap on the GPU (different
+ *   streams, no ordering between them) race on the array: order them.
+ *   A pipeline timeout on this path is recorded in the array, not in the flag
+ *   that rs_get_last_device_error reads. */
+int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                           const void* gamma, const void* beta, void* hidden, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* rs_status_string(int status);
 
