@@ -8,11 +8,13 @@ One step = one pass of the whole path over one batch of the workload (every
 stage for the chained UMT-L workload). Prints one JSON line on rank 0.
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on
-the launch stream with an L2 flush (a 256 MiB write, outside the events)
-before it; a barrier and a device synchronise on both sides of the loop; the
-max over ranks. Per-kernel durations for the roofline come from a second
-event-timed loop over the same kernels launched one step-level entry point at a
-time. `--impl reference` times the fp64 CPU oracle instead (rank 0 only).
+the launch stream with an L2 flush before it (outside the events: a 256 MiB
+write, then a 256 MiB read of a second buffer so that the write's dirty lines
+are written back before the step starts); a barrier and a device synchronise
+on both sides of the loop; the max over ranks. Per-kernel durations for the
+roofline come from a second event-timed loop over the same kernels, launched
+one step-level entry point (one kernel) at a time. `--impl reference` times
+the fp64 CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -36,7 +38,11 @@ from workloads import WORKLOADS, make_inputs  # noqa: E402
 METRIC = "pruned-MLP-block tokens/sec at 1 B200; % of bf16 tensor peak; select+gather GB/s"
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
-KERNELS_PER_STAGE = 5  # LN stats, fc1, fc2, select, gather
+def kernels_per_step(wl) -> int:
+    """Kernels rs_block_forward launches per stage: LN prep (statistics + weight
+    fold), fc1, fc2, then one fused select+gather kernel (L <= 256) or select and
+    gather (longer L)."""
+    return sum(4 if wl.stage_L(s) <= 256 else 5 for s in range(wl.stages))
 
 
 def load_peaks():
@@ -141,11 +147,13 @@ def max_over_ranks(v: float, world: int) -> float:
 
 # ----------------------------------------------------------------------------- oracle leg
 def oracle_rate(wl, seed: int, budget_s: float):
-    """Oracle tokens/s on a bounded sample of the workload (host cores)."""
+    """Oracle tokens/s on a bounded sample of the workload (host cores): whole
+    samples (all stages) one at a time, cycling over the batch, until the budget
+    is spent (at least one sample)."""
     import oracle
     from threadpoolctl import threadpool_info
 
-    inp = make_inputs(wl, seed=seed, batch=min(wl.B, 64))
+    inp = make_inputs(wl, seed=seed)
 
     def w64(w):
         f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
@@ -153,11 +161,11 @@ def oracle_rate(wl, seed: int, budget_s: float):
                     beta=f(w.beta))
 
     weights = [w64(w) for w in inp.weights]
-    x_all = inp.x.to(torch.float64).numpy()
     t0 = time.time()
     done_tokens, samples = 0, 0
-    while samples < x_all.shape[0] and (time.time() - t0) < budget_s:
-        x = x_all[samples:samples + 1]
+    while samples == 0 or (time.time() - t0) < budget_s:
+        b = samples % wl.B
+        x = inp.x[b:b + 1].to(torch.float64).numpy()
         for s in range(wl.stages):
             yk, _, _, _ = oracle.block_forward(x, keep_k=wl.keep_k[s], **weights[s])
             done_tokens += x.shape[1]
@@ -185,7 +193,7 @@ def main():
     config = {"workload": wl.name, "B": wl.B, "L": wl.L, "C": wl.C, "H": wl.H,
               "keep_k": list(wl.keep_k), "stages": wl.stages,
               "tokens_per_step": tokens_per_step, "parallelism": f"replicas{world}",
-              "l2": "flushed between timed steps (256 MiB write)"}
+              "l2": "flushed before every timed step: 256 MiB write + 256 MiB read"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -225,7 +233,12 @@ def main():
              torch.empty(wl.B, k + 1, dtype=torch.int32, device=dev),
              torch.empty(wl.B, wl.stage_L(s), dtype=torch.float32, device=dev))
             for s, k in enumerate(wl.keep_k)]
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def l2_flush():
+        flush_w.zero_()
+        flush_r.sum()
 
     def step(x0):
         xs = x0
@@ -236,7 +249,7 @@ def main():
     clocks = ClockSampler(local)
     clocks.start()
     for _ in range(args.warmup):
-        flush.zero_()
+        l2_flush()
         step(x)
     torch.cuda.synchronize()
     assert rs.rs_get_last_device_error() == 0
@@ -246,7 +259,7 @@ def main():
     torch.cuda.synchronize()
     clocks.mark_start = time.time()
     for i in range(args.steps):
-        flush.zero_()
+        l2_flush()
         ev[i][0].record(stream)
         step(x)
         ev[i][1].record(stream)
@@ -260,54 +273,57 @@ def main():
     ms_per_step = total_ms / args.steps
     value = world * tokens_per_step * args.steps / (total_ms / 1e3)
 
-    # ---- per-kernel breakdown (same kernels, one step-level entry point at a time)
-    kt = {"fc1": [], "fc2": [], "select": [], "gather": []}
+    # ---- per-kernel breakdown (the same kernels, one step-level entry point each)
+    names = ("stats", "fold", "fc1", "fc2", "select_gather")
     M0 = wl.tokens(0)
+    np_ = rs.rs_num_partials(wl.C)
+    stats = torch.empty(M0, 2, dtype=torch.float32, device=dev)
+    Wg = torch.empty(wl.H, wl.C, dtype=torch.bfloat16, device=dev)
+    colG = torch.empty(wl.H, dtype=torch.float32, device=dev)
+    colC = torch.empty(wl.H, dtype=torch.float32, device=dev)
     hid = torch.empty(M0 * wl.H, dtype=torch.bfloat16, device=dev)
     ybuf = torch.empty(M0 * wl.C, dtype=torch.bfloat16, device=dev)
-    np_ = rs.rs_num_partials(wl.C)
     pbuf = torch.empty(M0 * np_, dtype=torch.float32, device=dev)
     nrep = max(10, min(args.steps, 200))
     recs = []
     for i in range(nrep):
-        flush.zero_()
+        l2_flush()
         xs = x
         for s, k in enumerate(wl.keep_k):
             L_s = wl.stage_L(s)
             M = wl.B * L_s
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
             x2 = xs.reshape(M, wl.C)
+            st2 = stats[:M]
             h2 = hid[: M * wl.H].view(M, wl.H)
             y2 = ybuf[: M * wl.C].view(M, wl.C)
             p2 = pbuf[: M * np_].view(M, np_)
             e[0].record(stream)
-            rs.rs_ln_fc1_gelu(x2, W[s][0], W[s][1], W[s][4], W[s][5], hidden=h2, stream=stream)
+            rs.rs_ln_stats(x2, stats=st2, stream=stream)
             e[1].record(stream)
-            rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
+            rs.rs_ln_fold(W[s][0], W[s][1], W[s][4], W[s][5], Wg, colG, colC, stream=stream)
             e[2].record(stream)
-            rs.rs_select_topk(p2, wl.B, L_s, k, scores=outs[s][2], kept_idx=outs[s][1],
-                              stream=stream)
+            rs.rs_fc1_gelu_folded(x2, st2, Wg, colG, colC, hidden=h2, stream=stream)
             e[3].record(stream)
-            rs.rs_gather_rows(y2.view(wl.B, L_s, wl.C), outs[s][1], k, y_kept=outs[s][0],
-                              stream=stream)
+            rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
             e[4].record(stream)
+            rs.rs_select_gather(p2, y2.view(wl.B, L_s, wl.C), k, scores=outs[s][2],
+                                kept_idx=outs[s][1], y_kept=outs[s][0], stream=stream)
+            e[5].record(stream)
             recs.append((s, e))
             xs = outs[s][0]
     torch.cuda.synchronize()
     per_stage = {}
     for s, e in recs:
-        d = per_stage.setdefault(s, {"fc1": [], "fc2": [], "select": [], "gather": []})
-        d["fc1"].append(e[0].elapsed_time(e[1]))
-        d["fc2"].append(e[1].elapsed_time(e[2]))
-        d["select"].append(e[2].elapsed_time(e[3]))
-        d["gather"].append(e[3].elapsed_time(e[4]))
+        d = per_stage.setdefault(s, {n: [] for n in names})
+        for j, n in enumerate(names):
+            d[n].append(e[j].elapsed_time(e[j + 1]))
     gemm_flops = {s: 2.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages)}
     fc_ms = {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage) for n in ("fc1", "fc2")}
     dominant = max(fc_ms, key=fc_ms.get)
     flops = sum(gemm_flops.values())
     achieved_tf = flops / (fc_ms[dominant] / 1e3) / 1e12
-    sel_ms = sum(statistics.mean(per_stage[s]["select"]) + statistics.mean(per_stage[s]["gather"])
-                 for s in per_stage)
+    sel_ms = sum(statistics.mean(per_stage[s]["select_gather"]) for s in per_stage)
     sg_bytes = 0
     for s, k in enumerate(wl.keep_k):
         M = wl.tokens(s)
@@ -326,7 +342,7 @@ def main():
     e2e_ev = []
     barrier(world)
     for i in range(n_e2e):
-        flush.zero_()
+        l2_flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         x_d.copy_(x_h, non_blocking=True)
@@ -345,8 +361,8 @@ def main():
     if rank == 0 and args.cpu_budget > 0:
         r, n, dt, thr = oracle_rate(wl, 0, args.cpu_budget)
         cpu = {"value": r, "unit": UNIT, "cores": thr, "kind": "oracle",
-               "sample": f"{n} of {wl.B} samples of {wl.name} (all stages) in {dt:.1f} s "
-                         f"on the host, fp64 numpy/BLAS"}
+               "sample": f"{n} samples of {wl.name} (all stages, one sample at a time) in "
+                         f"{dt:.1f} s on the host, fp64 numpy/BLAS"}
 
     peak_tf = peaks["bf16"]
     line = {
@@ -362,13 +378,13 @@ def main():
         "block_tflops": block_flops / (ms_per_step / 1e3) / 1e12,
         "block_frac_of_bf16_peak": block_flops / (ms_per_step / 1e3) / 1e12 / peak_tf,
         "kernel_ms": {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage)
-                      for n in ("fc1", "fc2", "select", "gather")},
+                      for n in names},
         "select_gather": {"GBps": sg_gbs, "frac_hbm": sg_gbs / peaks["hbm"],
                           "bytes": sg_bytes, "ms": sel_ms},
         "images_per_s": world * wl.B / (ms_per_step / 1e3),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": KERNELS_PER_STAGE * wl.stages * args.steps,
+        "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
     }

@@ -8,15 +8,18 @@ from .rs import (  # noqa: F401
     lib,
     rs_block_forward,
     rs_fc2_residual_shift,
+    rs_fc1_gelu_folded,
     rs_gather_rows,
     rs_gelu_apply,
     rs_get_last_device_error,
     rs_ln_fc1_gelu,
+    rs_ln_fold,
     rs_ln_fc1_gelu_noalloc,
     rs_ln_fc1_gelu_staged,
     rs_ln_stats,
     rs_num_partials,
     rs_release_workspace,
+    rs_select_gather,
     rs_select_topk,
     rs_workspace_bytes,
     status_string,

@@ -154,14 +154,15 @@ int check_rows(int64_t M, int C, int H) {
     }                                                       \
   } while (0)
 
-// LN statistics, then fc1 with the LayerNorm folded into the GEMM (default) or
-// staged into the A operand by LN warps (staged = true). `ws` holds the fc1
-// part of the workspace layout for these sizes.
+// LN statistics (and, for the folded LN, the weight fold in the same launch),
+// then fc1 with the LayerNorm folded into the GEMM (default) or staged into the
+// A operand by LN warps (staged = true). `ws` holds the fc1 part of the
+// workspace layout for these sizes. The first launch follows the stream's
+// previous work normally; the GEMM is a programmatic dependent launch.
 int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, const void* b1,
             const void* gamma, const void* beta, uint8_t* ws, const WsLayout& w, void* hidden,
             bool staged, cudaStream_t s) {
   float* stats = reinterpret_cast<float*>(ws + w.stats);
-  RS_CUDA(rs::launch_ln_stats(x, M, C, stats, st.num_sms, s));
   const int bn = rs::fc1_block_n(H);
   rs::MlpParams p{};
   p.M = M;
@@ -175,6 +176,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   p.timeout_ns = rs::kDefaultTimeoutNs;
   const void* wB = W1;
   if (staged) {
+    RS_CUDA(rs::launch_ln_stats(x, M, C, stats, st.num_sms, s));
     p.ln_gamma = static_cast<const __nv_bfloat16*>(gamma);
     p.ln_beta = static_cast<const __nv_bfloat16*>(beta);
     p.bias = static_cast<const __nv_bfloat16*>(b1);
@@ -182,7 +184,8 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
     void* wg = ws + w.wg;
     float* colg = reinterpret_cast<float*>(ws + w.colg);
     float* colc = reinterpret_cast<float*>(ws + w.colc);
-    RS_CUDA(rs::launch_ln_fold(W1, gamma, beta, b1, H, C, wg, colg, colc, st.num_sms, s));
+    RS_CUDA(rs::launch_ln_prep(x, M, C, stats, W1, gamma, beta, b1, H, wg, colg, colc, st.num_sms,
+                               s));
     p.colG = colg;
     p.colC = colc;
     wB = wg;
@@ -191,16 +194,17 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, wB, C, H, bn));
   RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
-  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, st.num_sms, s));
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, st.num_sms, s, /*pdl=*/true));
   return RS_OK;
 }
 
 int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H, const void* W2,
-            const void* b2, void* y, float* partials, cudaStream_t s) {
+            const void* b2, void* y, float* partials, cudaStream_t s, bool pdl = false) {
   const int bn = rs::fc2_block_n(C);
-  CUtensorMap tmH, tmW;
+  CUtensorMap tmH, tmW, tmY;
   RS_TRY(make_tmap(&tmH, hidden, H, M, 128));
   RS_TRY(make_tmap(&tmW, W2, H, C, bn));
+  RS_TRY(make_tmap(&tmY, y, C, M, 32, 32));
   rs::MlpParams p{};
   p.M = M;
   p.N = C;
@@ -214,7 +218,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.num_partials = 2 * p.n_blocks;
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
-  RS_CUDA(rs::launch_fc2(tmH, tmW, p, bn, st.num_sms, s));
+  RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, st.num_sms, s, pdl));
   return RS_OK;
 }
 
@@ -289,6 +293,59 @@ int rs_ln_fc1_gelu_staged(const void* x, int M, int C, int H, const void* W1, co
   return ln_fc1_gelu(x, M, C, H, W1, b1, gamma, beta, hidden, true, stream);
 }
 
+int rs_ln_fold(const void* W1, const void* b1, const void* gamma, const void* beta, int C, int H,
+               void* Wg, float* colG, float* colC, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  if (!W1 || !b1 || !gamma || !beta || !Wg || !colG || !colC) return RS_ERR_NULL;
+  if (!al16(W1) || !al16(gamma) || !al16(beta) || !al16(Wg) || !al4(colG) || !al4(colC))
+    return RS_ERR_ALIGN;
+  int num_sms = 148;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevState* st = nullptr;
+    RS_TRY(dev_state(&st));
+    num_sms = st->num_sms;
+  }
+  RS_CUDA(rs::launch_ln_fold(W1, gamma, beta, b1, H, C, Wg, colG, colC, num_sms,
+                             static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const float* colG,
+                       const float* colC, int M, int C, int H, void* hidden, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (M == 0) return RS_OK;
+  if (!x || !stats || !Wg || !colG || !colC || !hidden) return RS_ERR_NULL;
+  if (!al16(x) || !al8(stats) || !al16(Wg) || !al16(colG) || !al16(colC) || !al16(hidden))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  const int bn = rs::fc1_block_n(H);
+  CUtensorMap tmX, tmW, tmHid;
+  RS_TRY(make_tmap(&tmX, x, C, M, 128));
+  RS_TRY(make_tmap(&tmW, Wg, C, H, bn));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
+  rs::MlpParams p{};
+  p.M = M;
+  p.N = H;
+  p.K = C;
+  p.n_blocks = H / bn;
+  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.stats = reinterpret_cast<const float2*>(stats);
+  p.colG = colG;
+  p.colC = colC;
+  p.out = static_cast<__nv_bfloat16*>(hidden);
+  p.err = st->err;
+  p.timeout_ns = rs::kDefaultTimeoutNs;
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, st->num_sms,
+                         static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
 int rs_gelu_apply(const float* z, float* out, int n, void* stream) {
   if (n < 0) return RS_ERR_SHAPE;
   if (n == 0) return RS_OK;
@@ -325,6 +382,29 @@ int rs_select_topk(const float* partials, int num_partials, int B, int L, int ke
   if (!al4(partials) || !al4(scores) || !al4(kept_idx)) return RS_ERR_ALIGN;
   RS_CUDA(rs::launch_select(partials, num_partials, B, L, keep_k, scores, kept_idx,
                             static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_select_gather(const float* partials, int num_partials, const void* y, int B, int L, int C,
+                     int keep_k, float* scores, int32_t* kept_idx, void* y_kept, void* stream) {
+  RS_TRY(check_width(C));
+  if (B < 0 || L < 1 || L > RS_MAX_L || num_partials < 1 || num_partials > 64)
+    return RS_ERR_SHAPE;
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, num_partials));
+  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  if (B == 0) return RS_OK;
+  if (!partials || !y || !scores || !kept_idx || !y_kept) return RS_ERR_NULL;
+  if (!al4(partials) || !al16(y) || !al4(scores) || !al4(kept_idx) || !al16(y_kept))
+    return RS_ERR_ALIGN;
+  int num_sms = 148;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevState* st = nullptr;
+    RS_TRY(dev_state(&st));
+    num_sms = st->num_sms;
+  }
+  RS_CUDA(rs::launch_select_gather(partials, num_partials, y, B, L, C, keep_k, scores, kept_idx,
+                                   y_kept, num_sms, static_cast<cudaStream_t>(stream)));
   return RS_OK;
 }
 
@@ -379,9 +459,9 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
   const int np = 2 * C / rs::fc2_block_n(C);
 
   RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
-  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s));
-  RS_CUDA(rs::launch_select(partials, np, B, L, keep_k, scores, kept_idx, s));
-  RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k, y_kept, st->num_sms, s));
+  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s, /*pdl=*/true));
+  RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, scores, kept_idx, y_kept,
+                                   st->num_sms, s, /*pdl=*/true));
   return RS_OK;
 }
 

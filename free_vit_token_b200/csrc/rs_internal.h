@@ -18,6 +18,25 @@ constexpr int kEpiResidShift = 1;        // fc2 epilogue: + b2, residual, shift 
 constexpr int kEpiGeluFold = 2;          // fc1 epilogue: folded LN (mean, rstd, G, cb), erf-GELU
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // one pipeline wait: 4 s
 
+// Launches `kern` on `stream`; with `pdl` the launch may begin while the
+// previous kernel in the stream is still running (every kernel of this library
+// waits for its predecessor with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 struct MlpParams {
   int M, N, K;                    // output rows, output columns, reduction length
   int n_blocks, num_tiles;        // N / BN, ceil(M / 128) * n_blocks
@@ -39,18 +58,28 @@ size_t mlp_smem_bytes(int bn, bool ln, int epi, int K);
 int fc1_block_n(int H);
 int fc2_block_n(int C);
 cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl = false);
 cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,
                            int H, int C, void* Wg, float* colG, float* colC, int num_sms,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool pdl = false);
+// LN statistics of x' and the fold of gamma, beta into W1, in one launch.
+cudaError_t launch_ln_prep(const void* x, int M, int C, float* stats, const void* W1,
+                           const void* gamma, const void* beta, const void* b1, int H, void* Wg,
+                           float* colG, float* colC, int num_sms, cudaStream_t stream,
+                           bool pdl = false);
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s);
+                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s,
+                       bool pdl = false);
 cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream);
-cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p,
-                       int bn, int num_sms, cudaStream_t s);
+cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
+                       const MlpParams& p, int bn, int num_sms, cudaStream_t s, bool pdl = false);
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
-                          float* scores, int32_t* kept_idx, cudaStream_t stream);
+                          float* scores, int32_t* kept_idx, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
-                          void* y_kept, int num_sms, cudaStream_t stream);
+                          void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);
+// Selection then gather: one fused kernel for L <= 256, else the two kernels above.
+cudaError_t launch_select_gather(const float* partials, int num_partials, const void* y, int B,
+                                 int L, int C, int keep_k, float* scores, int32_t* kept_idx,
+                                 void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);
 
 }  // namespace rs

@@ -36,13 +36,13 @@ __device__ __forceinline__ void load_row(const uint4* __restrict__ xr, int lane,
 }
 
 // Persistent: each warp walks rows with a grid-wide stride and keeps the next
-// row's loads in flight while it reduces the current one.
+// row's loads in flight while it reduces the current one. `gw0`/`nw` are this
+// warp's index and the warp count of the part of the grid doing this work.
 template <int VPL>
-__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int M,
-                                                       int C, float2* __restrict__ stats) {
+__device__ __forceinline__ void ln_stats_body(const __nv_bfloat16* __restrict__ x, int M, int C,
+                                              float2* __restrict__ stats, int gw0, int nw) {
   const int lane = threadIdx.x & 31;
-  const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
-  int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  int row = gw0;
   const int nvec = C >> 3;
   const float inv_c = 1.0f / static_cast<float>(C);
   uint4 cur[VPL], nxt[VPL];
@@ -82,13 +82,22 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __re
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(256)
-    ln_fold_kernel(const __nv_bfloat16* __restrict__ W1, const __nv_bfloat16* __restrict__ gamma,
-                   const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ b1,
-                   int H, int C, __nv_bfloat16* __restrict__ Wg, float* __restrict__ colG,
-                   float* __restrict__ colC) {
+__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int M,
+                                                       int C, float2* __restrict__ stats) {
+  pdl_trigger();
+  pdl_wait();
+  ln_stats_body<VPL>(x, M, C, stats, static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5),
+                     static_cast<int>((gridDim.x * blockDim.x) >> 5));
+}
+
+template <int VPL>
+__device__ __forceinline__ void ln_fold_body(const __nv_bfloat16* __restrict__ W1,
+                                             const __nv_bfloat16* __restrict__ gamma,
+                                             const __nv_bfloat16* __restrict__ beta,
+                                             const __nv_bfloat16* __restrict__ b1, int H, int C,
+                                             __nv_bfloat16* __restrict__ Wg, float* __restrict__ colG,
+                                             float* __restrict__ colC, int gw0, int nw) {
   const int lane = threadIdx.x & 31;
-  const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
   const int nvec = C >> 3;
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
@@ -99,7 +108,7 @@ __global__ void __launch_bounds__(256)
     gv[i] = idx < nvec ? __ldg(g4 + idx) : make_uint4(0, 0, 0, 0);
     bv[i] = idx < nvec ? __ldg(b4 + idx) : make_uint4(0, 0, 0, 0);
   }
-  for (int j = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); j < H; j += nw) {
+  for (int j = gw0; j < H; j += nw) {
     const uint4* wr = reinterpret_cast<const uint4*>(W1 + static_cast<size_t>(j) * C);
     uint4* out = reinterpret_cast<uint4*>(Wg + static_cast<size_t>(j) * C);
     float gs = 0.f, cs = 0.f;
@@ -132,44 +141,106 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
-                            cudaStream_t stream) {
+template <int VPL>
+__global__ void __launch_bounds__(256)
+    ln_fold_kernel(const __nv_bfloat16* __restrict__ W1, const __nv_bfloat16* __restrict__ gamma,
+                   const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ b1,
+                   int H, int C, __nv_bfloat16* __restrict__ Wg, float* __restrict__ colG,
+                   float* __restrict__ colC) {
+  pdl_trigger();
+  pdl_wait();
+  ln_fold_body<VPL>(W1, gamma, beta, b1, H, C, Wg, colG, colC,
+                    static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5),
+                    static_cast<int>((gridDim.x * blockDim.x) >> 5));
+}
+
+// Both in one grid: the first `stats_blocks` blocks compute statistics, the rest fold.
+template <int VPL>
+__global__ void __launch_bounds__(256)
+    ln_prep_kernel(const __nv_bfloat16* __restrict__ x, int M, float2* __restrict__ stats,
+                   int stats_blocks, const __nv_bfloat16* __restrict__ W1,
+                   const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
+                   const __nv_bfloat16* __restrict__ b1, int H, int C,
+                   __nv_bfloat16* __restrict__ Wg, float* __restrict__ colG,
+                   float* __restrict__ colC) {
+  pdl_trigger();
+  pdl_wait();
+  const int wpb = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  if (static_cast<int>(blockIdx.x) < stats_blocks) {
+    ln_stats_body<VPL>(x, M, C, stats, blockIdx.x * wpb + w, stats_blocks * wpb);
+  } else {
+    const int fb = blockIdx.x - stats_blocks;
+    ln_fold_body<VPL>(W1, gamma, beta, b1, H, C, Wg, colG, colC, fb * wpb + w,
+                      (gridDim.x - stats_blocks) * wpb);
+  }
+}
+
+static int stats_blocks_for(int M, int num_sms) {
   const int warps = (M + 1) / 2;  // two rows per warp on average keeps loads in flight
   int blocks = (warps + 7) / 8;
   if (blocks > num_sms * 8) blocks = num_sms * 8;
-  if (blocks < 1) blocks = 1;
+  return blocks < 1 ? 1 : blocks;
+}
+static int fold_blocks_for(int H, int num_sms) {
+  int blocks = (H + 7) / 8;
+  if (blocks > num_sms * 4) blocks = num_sms * 4;
+  return blocks < 1 ? 1 : blocks;
+}
+
+cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
+                            cudaStream_t stream, bool pdl) {
+  const int blocks = stats_blocks_for(M, num_sms);
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* sp = reinterpret_cast<float2*>(stats);
-  if (C <= 256)
-    ln_stats_kernel<1><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
-  else if (C <= 512)
-    ln_stats_kernel<2><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
-  else if (C <= 1024)
-    ln_stats_kernel<4><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
-  else
-    ln_stats_kernel<8><<<blocks, 256, 0, stream>>>(xp, M, C, sp);
-  return cudaGetLastError();
+  if (C <= 256) return launch(ln_stats_kernel<1>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  if (C <= 512) return launch(ln_stats_kernel<2>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  if (C <= 1024) return launch(ln_stats_kernel<4>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  return launch(ln_stats_kernel<8>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
 }
 
 cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,
                            int H, int C, void* Wg, float* colG, float* colC, int num_sms,
-                           cudaStream_t stream) {
-  int blocks = (H + 7) / 8;
-  if (blocks > num_sms * 4) blocks = num_sms * 4;
+                           cudaStream_t stream, bool pdl) {
+  const int blocks = fold_blocks_for(H, num_sms);
   const auto* w = static_cast<const __nv_bfloat16*>(W1);
   const auto* g = static_cast<const __nv_bfloat16*>(gamma);
   const auto* b = static_cast<const __nv_bfloat16*>(beta);
   const auto* bb = static_cast<const __nv_bfloat16*>(b1);
   auto* o = static_cast<__nv_bfloat16*>(Wg);
   if (C <= 256)
-    ln_fold_kernel<1><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
-  else if (C <= 512)
-    ln_fold_kernel<2><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
-  else if (C <= 1024)
-    ln_fold_kernel<4><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
-  else
-    ln_fold_kernel<8><<<blocks, 256, 0, stream>>>(w, g, b, bb, H, C, o, colG, colC);
-  return cudaGetLastError();
+    return launch(ln_fold_kernel<1>, blocks, 256, 0, stream, pdl, w, g, b, bb, H, C, o, colG, colC);
+  if (C <= 512)
+    return launch(ln_fold_kernel<2>, blocks, 256, 0, stream, pdl, w, g, b, bb, H, C, o, colG, colC);
+  if (C <= 1024)
+    return launch(ln_fold_kernel<4>, blocks, 256, 0, stream, pdl, w, g, b, bb, H, C, o, colG, colC);
+  return launch(ln_fold_kernel<8>, blocks, 256, 0, stream, pdl, w, g, b, bb, H, C, o, colG, colC);
+}
+
+cudaError_t launch_ln_prep(const void* x, int M, int C, float* stats, const void* W1,
+                           const void* gamma, const void* beta, const void* b1, int H, void* Wg,
+                           float* colG, float* colC, int num_sms, cudaStream_t stream, bool pdl) {
+  const int sb = stats_blocks_for(M, num_sms);
+  const int fb = fold_blocks_for(H, num_sms);
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  auto* sp = reinterpret_cast<float2*>(stats);
+  const auto* w = static_cast<const __nv_bfloat16*>(W1);
+  const auto* g = static_cast<const __nv_bfloat16*>(gamma);
+  const auto* b = static_cast<const __nv_bfloat16*>(beta);
+  const auto* bb = static_cast<const __nv_bfloat16*>(b1);
+  auto* o = static_cast<__nv_bfloat16*>(Wg);
+  const dim3 grid(sb + fb);
+  if (C <= 256)
+    return launch(ln_prep_kernel<1>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+                  colG, colC);
+  if (C <= 512)
+    return launch(ln_prep_kernel<2>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+                  colG, colC);
+  if (C <= 1024)
+    return launch(ln_prep_kernel<4>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+                  colG, colC);
+  return launch(ln_prep_kernel<8>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+                colG, colC);
 }
 
 }  // namespace rs

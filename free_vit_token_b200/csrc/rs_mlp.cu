@@ -40,12 +40,22 @@ constexpr int kCtrlBytes = 512;                 // barriers, TMEM slot, abort fl
 constexpr int kEpiBoxBytes = 32 * 32 * 2;       // one warp's 32 x 32 bf16 output box
 constexpr uint32_t kTmemCols = 512;
 
+constexpr int kVecMaxBytes = 2 * 256 * 4;       // one tile's column vectors (fold: G and cb)
+
 __host__ __device__ constexpr int stage_bytes(int bn) { return kAStageBytes + bn * kBK * 2; }
+// Per-tile column vectors the epilogue reads: the folded-LN G and cb (fp32) or
+// the bias (bf16), for BN columns; double-buffered with the accumulator.
+__host__ __device__ constexpr int vec_bytes(int bn, int epi) {
+  return epi == kEpiGeluFold ? 2 * bn * 4 : bn * 2;
+}
+__host__ __device__ constexpr int vec_stride(int bn, int epi) {
+  return (vec_bytes(bn, epi) + 127) / 128 * 128;
+}
 __host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
   // alignment slack + control block + gamma/beta (bf16, up to RS_MAX_C each) +
-  // the fc1 epilogue's per-warp output boxes
-  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) +
-         (epi != kEpiResidShift ? kNumEpiWarps * kEpiBoxBytes : 0);
+  // the epilogue's per-warp output boxes + two tiles' column vectors
+  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + kNumEpiWarps * kEpiBoxBytes +
+         2 * kVecMaxBytes;
 }
 __host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
   return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn) > 6
@@ -56,7 +66,7 @@ __host__ __device__ constexpr int num_threads(bool ln) { return (ln ? 16 : 12) *
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K) {
   return 1024 + static_cast<size_t>(num_stages(bn, ln, epi)) * stage_bytes(bn) +
-         (epi != kEpiResidShift ? kNumEpiWarps * kEpiBoxBytes : 0) + kCtrlBytes +
+         kNumEpiWarps * kEpiBoxBytes + 2 * vec_stride(bn, epi) + kCtrlBytes +
          (ln ? 4 * static_cast<size_t>(K) : 0);
 }
 
@@ -118,8 +128,9 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   constexpr int kBStageBytes = BN * kBK * 2;
   constexpr int STAGES = num_stages(BN, LN_A, EPI);
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN);
-  constexpr bool kGeluOut = EPI != kEpiResidShift;  // fc1: GELU, TMA-store boxes
-  constexpr int kOutBytes = kGeluOut ? kNumEpiWarps * kEpiBoxBytes : 0;
+  constexpr int kOutBytes = kNumEpiWarps * kEpiBoxBytes;
+  constexpr int kVecBytes = vec_bytes(BN, EPI);
+  constexpr int kVecStride = vec_stride(BN, EPI);
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(2 * BN <= static_cast<int>(kTmemCols), "TMEM double buffer");
   static_assert(STAGES >= 2, "pipeline depth");
@@ -130,15 +141,19 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kAStageBytes;
   uint8_t* sOut = sB + STAGES * kBStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kOutBytes);
+  uint8_t* sVec = sOut + kOutBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sVec + 2 * kVecStride);
   uint64_t* empty = full + STAGES;
   uint64_t* aready = empty + STAGES;
   uint64_t* tfull = aready + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* vfull = tempty + 2;
+  uint64_t* vempty = vfull + 2;
+  uint64_t* drain = vempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  __nv_bfloat16* s_gamma = reinterpret_cast<__nv_bfloat16*>(sOut + kOutBytes + kCtrlBytes);
+  __nv_bfloat16* s_gamma =
+      reinterpret_cast<__nv_bfloat16*>(sVec + 2 * kVecStride + kCtrlBytes);
   __nv_bfloat16* s_beta = s_gamma + p.K;
 
   const int warp = threadIdx.x >> 5;
@@ -154,6 +169,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kNumEpiWarps);
+      mbar_init(&vfull[a], 1);
+      mbar_init(&vempty[a], kNumEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -162,12 +179,16 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (kGeluOut) tma_prefetch_desc(&tmOut);
+    tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // Nothing above touched global memory: let the next kernel launch, then wait
+  // for the previous one to finish before reading anything it may have written.
+  pdl_trigger();
+  pdl_wait();
   if constexpr (LN_A) {
     const uint4* g = reinterpret_cast<const uint4*>(p.ln_gamma);
     const uint4* b = reinterpret_cast<const uint4*>(p.ln_beta);
@@ -187,11 +208,26 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int vacc = 0;
+      uint32_t vphase = 0;
       int pend[STAGES];
+      int vpend0 = -1, vpend1 = -1;
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) pend[s] = -1;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
         const int m_blk = tile / p.n_blocks, n_blk = tile % p.n_blocks;
+        // this tile's column vectors, into the buffer of the accumulator it will use
+        if (!wait_bounded(&vempty[vacc], vphase ^ 1u, wc)) break;
+        mbar_arrive_expect_tx(&vfull[vacc], kVecBytes);
+        uint8_t* vdst = sVec + vacc * kVecStride;
+        if constexpr (EPI == kEpiGeluFold) {
+          bulk_load(vdst, p.colG + n_blk * BN, BN * 4, &vfull[vacc]);
+          bulk_load(vdst + BN * 4, p.colC + n_blk * BN, BN * 4, &vfull[vacc]);
+        } else {
+          bulk_load(vdst, p.bias + n_blk * BN, BN * 2, &vfull[vacc]);
+        }
+        if (vacc == 0) vpend0 = static_cast<int>(vphase); else vpend1 = static_cast<int>(vphase);
+        if (++vacc == 2) { vacc = 0; vphase ^= 1u; }
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, wc)) { ok = false; break; }
@@ -205,10 +241,12 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         }
         if (!ok) break;
       }
-      // Every load this thread issued must land before the CTA may exit.
+      // Every copy this thread issued must land before the CTA may exit.
 #pragma unroll
       for (int s = 0; s < STAGES; ++s)
         if (pend[s] >= 0) wait_bounded(&full[s], static_cast<uint32_t>(pend[s]), wc, false);
+      if (vpend0 >= 0) wait_bounded(&vfull[0], static_cast<uint32_t>(vpend0), wc, false);
+      if (vpend1 >= 0) wait_bounded(&vfull[1], static_cast<uint32_t>(vpend1), wc, false);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -251,9 +289,12 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
     // Warp -> TMEM lane quadrant q (rows 32q..32q+31 of the tile) and one half
-    // of the BN columns; 32-column chunks, the TMEM load of chunk n+1 in flight
-    // while chunk n is processed. The accumulator is handed back to the MMA
-    // warp as soon as its last chunk is in registers.
+    // of the BN columns, in 32-column chunks: the TMEM load (and for fc2 the
+    // residual rows) of chunk n+1 are in flight while chunk n is processed. The
+    // accumulator goes back to the MMA warp as soon as its last chunk is in
+    // registers. Every chunk leaves through the warp's 32 x 32 output box
+    // (64-byte swizzle: 16-byte chunk j of row r at j ^ ((r >> 1) & 3)) and a
+    // TMA store; rows past M are clipped by the store.
     const int q = warp & 3;
     const int half = (warp - kEpiWarp0) >> 2;
     constexpr int kHalf = BN / 2;
@@ -265,16 +306,21 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int m_blk = tile / p.n_blocks, n_blk = tile % p.n_blocks;
       int ok = 1;
-      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, wc) ? 1 : 0;
+      if (lane == 0)
+        ok = (wait_bounded(&vfull[acc], acc_phase, wc) && wait_bounded(&tfull[acc], acc_phase, wc))
+                 ? 1
+                 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      mbar_try_wait(&tfull[acc], acc_phase);  // completed: acquire for every lane
+      mbar_try_wait(&vfull[acc], acc_phase);  // completed: acquire for every lane
+      mbar_try_wait(&tfull[acc], acc_phase);
       tc_fence_after_sync();
       const int row = m_blk * kBM + q * 32 + lane;
       const bool row_ok = row < p.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * kHalf);
       const int col0 = n_blk * BN + half * kHalf;
+      const uint32_t vec_u32 = smem_u32(sVec + acc * kVecStride);
       float part = 0.f;
       uint64_t nmu2 = 0, rs2 = 0;  // folded LN: (-mean, -mean), (rstd, rstd) of this row
       if constexpr (EPI == kEpiGeluFold) {
@@ -283,98 +329,108 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         nmu2 = f2pack(-st.x, -st.x);
         rs2 = f2pack(st.y, st.y);
       }
+      const uint4* xrow = reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.N + col0);
       uint32_t ra[32], rb[32];
+      uint4 xa[4] = {}, xb[4] = {};
       tmem_ld32_async(t_row, ra);
+      if constexpr (EPI == kEpiResidShift) {
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) xa[v] = __ldg(xrow + v);
+        }
+      }
 #pragma unroll
       for (int n = 0; n < NCH; ++n) {
         uint32_t(&r)[32] = (n & 1) ? rb : ra;
         uint32_t(&nx)[32] = (n & 1) ? ra : rb;
+        uint4(&xv)[4] = (n & 1) ? xb : xa;
+        uint4(&xn)[4] = (n & 1) ? xa : xb;
         tmem_wait_ld();
         reg_fence(r);
         if (n + 1 < NCH) {
           tmem_ld32_async(t_row + (n + 1) * 32, nx);
+          if constexpr (EPI == kEpiResidShift) {
+            if (row_ok) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) xn[v] = __ldg(xrow + (n + 1) * 4 + v);
+            }
+          }
         } else {
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
         const int c = n * 32;
+        const uint32_t cvec = (half * kHalf + c);  // column of this chunk within the tile
         uint32_t outw[16];
-        if constexpr (kGeluOut) {
-          if constexpr (EPI == kEpiGeluFold) {
-            // z = rstd * (acc - mean * G[col]) + cb[col], two columns per step
-            const ulonglong2* gp = reinterpret_cast<const ulonglong2*>(p.colG + col0 + c);
-            const ulonglong2* cp = reinterpret_cast<const ulonglong2*>(p.colC + col0 + c);
+        if constexpr (EPI == kEpiGeluFold) {
+          // z = rstd * (acc - mean * G[col]) + cb[col], two columns per step
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const ulonglong2 g4 = __ldg(gp + v), c4 = __ldg(cp + v);
-              const uint64_t za = ffma2(rs2, ffma2(nmu2, g4.x, f2pack(__uint_as_float(r[4 * v]),
-                                                                      __uint_as_float(r[4 * v + 1]))),
-                                        c4.x);
-              const uint64_t zb = ffma2(rs2, ffma2(nmu2, g4.y, f2pack(__uint_as_float(r[4 * v + 2]),
-                                                                      __uint_as_float(r[4 * v + 3]))),
-                                        c4.y);
-              const float2 ga = f2unpack(gelu2(za)), gb = f2unpack(gelu2(zb));
-              outw[2 * v] = pack_bf16x2(ga.x, ga.y);
-              outw[2 * v + 1] = pack_bf16x2(gb.x, gb.y);
-            }
-          } else {
-            const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
-            uint4 bv[4];
+          for (int v = 0; v < 8; ++v) {
+            const uint4 g4 = lds128(vec_u32 + (cvec + 4 * v) * 4);
+            const uint4 c4 = lds128(vec_u32 + BN * 4 + (cvec + 4 * v) * 4);
+            const uint64_t ga = (static_cast<uint64_t>(g4.y) << 32) | g4.x;
+            const uint64_t gb = (static_cast<uint64_t>(g4.w) << 32) | g4.z;
+            const uint64_t ca = (static_cast<uint64_t>(c4.y) << 32) | c4.x;
+            const uint64_t cb = (static_cast<uint64_t>(c4.w) << 32) | c4.z;
+            const uint64_t za = ffma2(
+                rs2, ffma2(nmu2, ga, f2pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]))),
+                ca);
+            const uint64_t zb = ffma2(
+                rs2,
+                ffma2(nmu2, gb, f2pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]))),
+                cb);
+            const float2 g0 = f2unpack(gelu2(za)), g1 = f2unpack(gelu2(zb));
+            outw[2 * v] = pack_bf16x2(g0.x, g0.y);
+            outw[2 * v + 1] = pack_bf16x2(g1.x, g1.y);
+          }
+        } else {
+          uint32_t bw[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) bv[v] = __ldg(bptr + v);
-            const uint32_t* bw = reinterpret_cast<const uint32_t*>(bv);
+          for (int v = 0; v < 4; ++v) {
+            const uint4 b4 = lds128(vec_u32 + (cvec + 8 * v) * 2);
+            bw[4 * v] = b4.x;
+            bw[4 * v + 1] = b4.y;
+            bw[4 * v + 2] = b4.z;
+            bw[4 * v + 3] = b4.w;
+          }
+          if constexpr (EPI == kEpiGelu) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float2 g = f2unpack(gelu2(f2pack(__uint_as_float(r[2 * e]) + bf16lo(bw[e]),
                                                      __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]))));
               outw[e] = pack_bf16x2(g.x, g.y);
             }
+          } else {
+            const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
+              const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
+              const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
+              outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
+              const float d0 = h0 - x0, d1 = h1 - x1;
+              part = fmaf(d0, d0, part);
+              part = fmaf(d1, d1, part);
+            }
           }
-          // Row `lane` of this warp's 32 x 32 output box, 64-byte swizzled
-          // (16-byte chunk j of row r at j ^ ((r >> 1) & 3)), then one TMA store.
-          if (lane == 0) bulk_wait_group_read0();
+        }
+        if (n + 1 == NCH) {
+          // the last chunk's column vectors are read: the buffer may be refilled
           __syncwarp();
+          if (lane == 0) mbar_arrive(&vempty[acc]);
+        }
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            sts128(box_u32 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
-                   make_uint4(outw[4 * j], outw[4 * j + 1], outw[4 * j + 2], outw[4 * j + 3]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmOut, box, col0 + c, m_blk * kBM + q * 32);
-            bulk_commit_group();
-          }
-        } else {
-          const uint4* bptr = reinterpret_cast<const uint4*>(p.bias + col0 + c);
-          uint4 bv[4];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) bv[v] = __ldg(bptr + v);
-          const uint32_t* bw = reinterpret_cast<const uint32_t*>(bv);
-          uint4 xv[4] = {};
-          const size_t off = static_cast<size_t>(row) * p.N + col0 + c;
-          if (row_ok) {
-            const uint4* xptr = reinterpret_cast<const uint4*>(p.resid + off);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) xv[v] = __ldg(xptr + v);
-          }
-          const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
-            const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-            const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-            outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
-            const float d0 = h0 - x0, d1 = h1 - x1;
-            part = fmaf(d0, d0, part);
-            part = fmaf(d1, d1, part);
-          }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + off);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
-          }
+        for (int j = 0; j < 4; ++j)
+          sts128(box_u32 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
+                 make_uint4(outw[4 * j], outw[4 * j + 1], outw[4 * j + 2], outw[4 * j + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmOut, box, col0 + c, m_blk * kBM + q * 32);
+          bulk_commit_group();
         }
       }
       if constexpr (EPI == kEpiResidShift) {
@@ -382,10 +438,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    if constexpr (kGeluOut) {
-      if (lane == 0) bulk_wait_group0();
-      __syncwarp();
-    }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
   } else if (LN_A && warp >= kLnWarp0) {
     // ------------------------------------------------------------ LayerNorm staging
     // The A stage holds raw x' (TMA, 128-byte swizzle: 16-byte chunk c of row r
@@ -469,15 +523,14 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
 template <int BN, bool LN_A, int EPI>
 static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                const CUtensorMap& tmOut, const MlpParams& p, int num_sms,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool pdl) {
   auto kern = mlp_gemm_kernel<BN, LN_A, EPI>;
   const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  kern<<<grid, num_threads(LN_A), smem, stream>>>(tmA, tmB, tmOut, p);
-  return cudaGetLastError();
+  return launch(kern, grid, num_threads(LN_A), smem, stream, pdl, tmA, tmB, tmOut, p);
 }
 
 int fc1_block_n(int H) { return H % 256 == 0 ? 256 : (H % 128 == 0 ? 128 : 64); }
@@ -486,28 +539,29 @@ int fc2_block_n(int C) {
 }
 
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s) {
+                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s,
+                       bool pdl) {
   if (staged_ln) {
     switch (bn) {
-      case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
-      case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
-      default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s);
+      case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+      case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+      default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
     }
   }
   switch (bn) {
-    case 256: return launch_gemm<256, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
-    case 128: return launch_gemm<128, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
-    default: return launch_gemm<64, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s);
+    case 256: return launch_gemm<256, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+    case 128: return launch_gemm<128, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+    default: return launch_gemm<64, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
   }
 }
 
-cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const MlpParams& p, int bn,
-                       int num_sms, cudaStream_t s) {
+cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
+                       const MlpParams& p, int bn, int num_sms, cudaStream_t s, bool pdl) {
   switch (bn) {
-    case 256: return launch_gemm<256, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
-    case 192: return launch_gemm<192, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
-    case 128: return launch_gemm<128, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
-    default: return launch_gemm<64, false, kEpiResidShift>(tmHid, tmW2, tmW2, p, num_sms, s);
+    case 256: return launch_gemm<256, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
+    case 192: return launch_gemm<192, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
+    case 128: return launch_gemm<128, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
+    default: return launch_gemm<64, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
   }
 }
 

@@ -3,19 +3,28 @@
 // Compression with FlashAttention", §3.1 pruned set x-tilde, §3.2 Eq. (4) and
 // "dropped the tokens having the lowest k scores").
 //
-// select: one CTA per sample. s_t = sqrt(sum_j P[t, j]) in fp32 (fixed order),
-//   then a 4-pass MSB-first radix select over the fp32 score bits of the patch
-//   tokens (non-negative floats order like their bit patterns) finds the k-th
-//   largest key T and how many keys equal to T are taken; an ordered ballot
-//   compaction then writes [0] ++ ascending(kept t): every key > T, and the
-//   keys == T with the lowest indices first.
-// gather: one warp per kept row, 16-byte vector loads and streaming stores.
+// Scores: s_t = sqrt(sum_j P[t, j]) in fp32, partials added left to right.
+// Selection compares fp32 score bits (non-negative floats order like their bit
+// patterns). Token u beats token t when key_u > key_t, or key_u == key_t and
+// u < t; the kept set is the k patch tokens (t = 1..L-1) beaten by fewer than k
+// others, written as [0] ++ ascending(kept t) -- CLS first, never ranked.
+//   * L <= 256: every thread holds one key and counts its beaters in one sweep
+//     over shared memory; an ordered ballot compaction follows.
+//   * longer L: a 4-pass MSB-first radix select finds the k-th largest key T
+//     and how many keys equal to T are kept; the ordered compaction keeps every
+//     key > T and the lowest-index keys == T.
+// Kernels: select (one CTA per sample), gather (warps share out each sample's
+// kept rows), and select+gather fused (B x S CTAs: each CTA selects its
+// sample's rows and copies every S-th kept row, so the copy spreads over the GPU).
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "rs_internal.h"
+#include "rs_ptx.cuh"
 
 namespace rs {
+
+constexpr int kRankMaxL = 256;
 
 // Exclusive prefix count of `flag` over the block in thread order; `total`
 // receives the block-wide count. Every thread of the block must call it.
@@ -44,42 +53,111 @@ __device__ __forceinline__ uint32_t block_exclusive_count(bool flag, uint32_t* s
   return res;
 }
 
-__global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ partials, int NP,
-                                                      int L, int k, float* __restrict__ scores,
-                                                      int32_t* __restrict__ kept) {
-  extern __shared__ uint32_t s_key[];  // [L] fp32 score bits
-  __shared__ uint32_t s_hist[256];
-  __shared__ uint32_t s_warp[33];
-  __shared__ uint32_t s_sel[2];
-  const int b = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
-  const int lane = tid & 31, warp = tid >> 5;
-
-  const float* P = partials + static_cast<size_t>(b) * L * NP;
-  for (int t = tid; t < L; t += nt) {
-    const float* pr = P + static_cast<size_t>(t) * NP;
-    float acc = 0.f;
-    for (int j = 0; j < NP; ++j) acc += pr[j];
-    const float s = sqrtf(acc);
-    scores[static_cast<size_t>(b) * L + t] = s;
-    s_key[t] = __float_as_uint(s);
+// Number of patch tokens u in 1..L-1 that beat key `key` of token t (t >= 1):
+// key_u >= key for u < t, key_u > key for u > t (u = t never counts). The sweep
+// is split at t so every key costs one compare. s_key holds L keys padded with
+// zeros to a multiple of 4: a zero pad lies above t and is never > key. The CLS
+// slot (u = 0 < t) counted exactly when key_0 >= key and is removed.
+__device__ __forceinline__ uint32_t count_beaters(const uint32_t* s_key, int L, uint32_t key,
+                                                  int t) {
+  const uint4* k4 = reinterpret_cast<const uint4*>(s_key);
+  const int q = (L + 3) >> 2;
+  const int qt = t >> 2;  // the quad holding t
+  uint32_t n = 0;
+#pragma unroll 4
+  for (int i = 0; i < qt; ++i) {
+    const uint4 v = k4[i];
+    n += (v.x >= key) + (v.y >= key) + (v.z >= key) + (v.w >= key);
   }
-  int32_t* out = kept + static_cast<size_t>(b) * (k + 1);
-  if (tid == 0) out[0] = 0;  // CLS: always kept, never ranked
-  if (k == 0) return;
-  __syncthreads();
+  {
+    const uint4 v = k4[qt];
+    const int r = t & 3;
+    n += r > 0 ? static_cast<uint32_t>(v.x >= key) : 0u;
+    n += r > 1 ? static_cast<uint32_t>(v.y >= key) : (r < 1 ? static_cast<uint32_t>(v.y > key) : 0u);
+    n += r > 2 ? static_cast<uint32_t>(v.z >= key) : (r < 2 ? static_cast<uint32_t>(v.z > key) : 0u);
+    n += r < 3 ? static_cast<uint32_t>(v.w > key) : 0u;
+  }
+#pragma unroll 4
+  for (int i = qt + 1; i < q; ++i) {
+    const uint4 v = k4[i];
+    n += (v.x > key) + (v.y > key) + (v.z > key) + (v.w > key);
+  }
+  return n - (s_key[0] >= key);  // CLS is never ranked
+}
 
+// Shared memory of one selecting CTA.
+struct SelSmem {
+  uint32_t* key;   // [roundup(L, 4)] score bits, zero padded
+  int32_t* kept;   // [k + 1] kept token list
+  uint32_t* warp;  // [33] block scan scratch
+  uint32_t* hist;  // [256] radix histogram
+  uint32_t* sel;   // [2] selected digit, count above it
+};
+
+__device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, uint32_t* s_hist,
+                                         uint32_t* s_sel) {
+  SelSmem s;
+  s.key = reinterpret_cast<uint32_t*>(dyn);
+  s.kept = reinterpret_cast<int32_t*>(dyn + ((L + 3) & ~3) * 4);
+  s.warp = s_warp;
+  s.hist = s_hist;
+  s.sel = s_sel;
+  return s;
+}
+
+// Scores of sample b from its partials into s.key (and to `scores` when given).
+__device__ __forceinline__ void load_keys(const float* __restrict__ partials, int NP, int L, int b,
+                                          float* __restrict__ scores, const SelSmem& s) {
+  const int Lpad = (L + 3) & ~3;
+  const float* P = partials + static_cast<size_t>(b) * L * NP;
+  for (int t = threadIdx.x; t < Lpad; t += blockDim.x) {
+    uint32_t key = 0;
+    if (t < L) {
+      const float* pr = P + static_cast<size_t>(t) * NP;
+      float acc = 0.f;
+      for (int j = 0; j < NP; ++j) acc += pr[j];
+      const float v = sqrtf(acc);
+      if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
+      key = __float_as_uint(v);
+    }
+    s.key[t] = key;
+  }
+  __syncthreads();
+}
+
+// The kept list of one sample into s.kept. Every thread of the block calls it;
+// it ends with a barrier, so s.kept is complete on return.
+__device__ void select_into_smem(int L, int k, const SelSmem& s) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s.kept[0] = 0;
+  if (k == 0) {
+    __syncthreads();
+    return;
+  }
+  if (L <= kRankMaxL && nt >= L) {
+    const int t = tid;
+    const uint32_t key = t < L ? s.key[t] : 0u;
+    const bool keep =
+        t >= 1 && t < L && count_beaters(s.key, L, key, t) < static_cast<uint32_t>(k);
+    uint32_t total;
+    const uint32_t pos = block_exclusive_count(keep, s.warp, total);
+    if (keep) s.kept[1 + pos] = t;
+    __syncthreads();
+    return;
+  }
   // Radix select of the k-th largest key among t = 1..L-1.
   uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += nt) s_hist[i] = 0;
+    for (int i = tid; i < 256; i += nt) s.hist[i] = 0;
     __syncthreads();
     for (int base = 1; base < L; base += nt) {
       const int t = base + tid;
-      const uint32_t u = t < L ? s_key[t] : 0u;
+      const uint32_t u = t < L ? s.key[t] : 0u;
       const bool cand = t < L && (u & mask) == prefix;
       const uint32_t digit = cand ? ((u >> shift) & 0xFFu) : 256u;
       const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], __popc(peers));
+      if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -87,7 +165,7 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        c[i] = s_hist[255 - 8 * lane - i];
+        c[i] = s.hist[255 - 8 * lane - i];
         sum += c[i];
       }
       uint32_t incl = sum;
@@ -101,8 +179,8 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (above + c[i] >= need) {
-            s_sel[0] = static_cast<uint32_t>(255 - 8 * lane - i);
-            s_sel[1] = above;
+            s.sel[0] = static_cast<uint32_t>(255 - 8 * lane - i);
+            s.sel[1] = above;
             break;
           }
           above += c[i];
@@ -110,98 +188,196 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
       }
     }
     __syncthreads();
-    prefix |= s_sel[0] << shift;
+    prefix |= s.sel[0] << shift;
     mask |= 0xFFu << shift;
-    need -= s_sel[1];
+    need -= s.sel[1];
     __syncthreads();
   }
   const uint32_t T = prefix;  // k-th largest key; `need` keys equal to T are kept
-
-  // Ordered compaction: ascending t.
   uint32_t eq_base = 0, out_base = 0;
   for (int base = 1; base < L; base += nt) {
     const int t = base + tid;
     const bool valid = t < L;
-    const uint32_t u = valid ? s_key[t] : 0u;
+    const uint32_t u = valid ? s.key[t] : 0u;
     const bool gt = valid && u > T;
     const bool eq = valid && u == T;
     uint32_t eq_tot, keep_tot;
-    const uint32_t eq_rank = eq_base + block_exclusive_count(eq, s_warp, eq_tot);
+    const uint32_t eq_rank = eq_base + block_exclusive_count(eq, s.warp, eq_tot);
     const bool keep = gt || (eq && eq_rank < need);
-    const uint32_t pos = out_base + block_exclusive_count(keep, s_warp, keep_tot);
-    if (keep) out[1 + pos] = t;
+    const uint32_t pos = out_base + block_exclusive_count(keep, s.warp, keep_tot);
+    if (keep) s.kept[1 + pos] = t;
     eq_base += eq_tot;
     out_base += keep_tot;
   }
+  __syncthreads();
 }
 
+__global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ partials, int NP,
+                                                      int L, int k, float* __restrict__ scores,
+                                                      int32_t* __restrict__ kept) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2];
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x;
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel);
+  load_keys(partials, NP, L, b, scores, s);
+  select_into_smem(L, k, s);
+  int32_t* out = kept + static_cast<size_t>(b) * (k + 1);
+  for (int i = threadIdx.x; i <= k; i += blockDim.x) out[i] = s.kept[i];
+}
+
+// Copies kept rows r = r_first, r_first + r_step, ... (r < k1) of sample b; a warp
+// moves kRows rows per iteration with all loads issued before the stores. Kept
+// indices come from shared memory (`rows` = the kept list) or from global
+// memory (`rows` = kept_idx [B, k1]); an index outside 0..L-1 gives a zero row.
+template <int VPL>
+__device__ __forceinline__ void copy_rows(const uint4* __restrict__ y, int L, int Cv, int b,
+                                          int k1, const int32_t* rows, bool rows_in_smem,
+                                          int r_first, int r_step, uint4* __restrict__ y_kept) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kRows = VPL >= 4 ? 1 : 4 / VPL;  // 16 registers of row data in flight
+  for (int r0 = r_first; r0 < k1; r0 += r_step * kRows) {
+    uint4 v[kRows][VPL];
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+      const int r = r0 + r_step * j;
+      if (r < k1) {
+        const int t = rows_in_smem ? rows[r] : __ldg(rows + static_cast<size_t>(b) * k1 + r);
+        if (t >= 0 && t < L) {
+          const uint4* src = y + (static_cast<size_t>(b) * L + t) * Cv;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i)
+            if (lane + 32 * i < Cv) v[j][i] = __ldg(src + lane + 32 * i);
+        } else {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) v[j][i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+      const int r = r0 + r_step * j;
+      if (r < k1) {
+        uint4* dst = y_kept + (static_cast<size_t>(b) * k1 + r) * Cv;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (lane + 32 * i < Cv) __stcs(dst + lane + 32 * i, v[j][i]);
+      }
+    }
+  }
+}
+
+// Fused: CTA (b, j0) of B x S selects sample b's kept rows and copies rows
+// j0, j0 + S, ... of them; CTA (b, 0) also writes scores and kept_idx.
+constexpr int kSelGatherThreads = 512;
+
+template <int VPL>
+__global__ void __launch_bounds__(kSelGatherThreads, 2) select_gather_kernel(
+    const float* __restrict__ partials, int NP, int L, int k, const uint4* __restrict__ y, int Cv,
+    int S, float* __restrict__ scores, int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2];
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x / S, j0 = blockIdx.x % S;
+  const bool writer = j0 == 0;
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel);
+  load_keys(partials, NP, L, b, writer ? scores : nullptr, s);
+  select_into_smem(L, k, s);
+  const int k1 = k + 1;
+  if (writer)
+    for (int i = threadIdx.x; i < k1; i += blockDim.x)
+      kept[static_cast<size_t>(b) * k1 + i] = s.kept[i];
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  copy_rows<VPL>(y, L, Cv, b, k1, s.kept, true, j0 + S * w, S * nw, y_kept);
+}
+
+// Standalone gather: the warps of the grid are shared out over the samples;
+// a sample's warps take its kept rows round robin.
 template <int VPL>
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ y, int L, int Cv,
                                                      const int32_t* __restrict__ kept, int k1,
-                                                     int rows_total, uint4* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
+                                                     int B, uint4* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
-  for (int row = gw; row < rows_total; row += nw) {
-    const int b = row / k1;
-    const int t = __ldg(kept + row);
-    uint4* dst = out + static_cast<size_t>(row) * Cv;
-    uint4 v[VPL];
-    if (t >= 0 && t < L) {
-      const uint4* src = y + (static_cast<size_t>(b) * L + t) * Cv;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int idx = lane + 32 * i;
-        if (idx < Cv) v[i] = __ldg(src + idx);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) v[i] = make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int idx = lane + 32 * i;
-      if (idx < Cv) __stcs(dst + idx, v[i]);
-    }
-  }
+  const int per_sample = nw / B > 0 ? nw / B : 1;
+  const int groups = nw / per_sample;
+  for (int b = gw / per_sample; b < B && gw < groups * per_sample; b += groups)
+    copy_rows<VPL>(y, L, Cv, b, k1, kept, false, gw % per_sample, per_sample, out);
+}
+
+static size_t select_smem(int L, int k) {
+  return static_cast<size_t>((L + 3) & ~3) * 4 + static_cast<size_t>(k + 1) * 4;
 }
 
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
-                          float* scores, int32_t* kept_idx, cudaStream_t stream) {
-  static bool attr_set = false;
-  const size_t smem = static_cast<size_t>(L) * sizeof(uint32_t);
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         RS_MAX_L * static_cast<int>(sizeof(uint32_t)));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+                          float* scores, int32_t* kept_idx, cudaStream_t stream, bool pdl) {
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L - 1)));
+  if (e != cudaSuccess) return e;
   int threads = ((L + 31) / 32) * 32;
-  if (threads > 1024) threads = 1024;
   if (threads < 64) threads = 64;
-  select_kernel<<<B, threads, smem, stream>>>(partials, num_partials, L, keep_k, scores, kept_idx);
-  return cudaGetLastError();
+  if (L > kRankMaxL) threads = 1024;
+  return launch(select_kernel, B, threads, select_smem(L, keep_k), stream, pdl, partials,
+                num_partials, L, keep_k, scores, kept_idx);
+}
+
+template <int VPL>
+static cudaError_t launch_gather_t(const void* y, int B, int L, int Cv, const int32_t* kept_idx,
+                                   int k1, void* y_kept, int blocks, cudaStream_t stream, bool pdl) {
+  return launch(gather_kernel<VPL>, blocks, 256, 0, stream, pdl, static_cast<const uint4*>(y), L,
+                Cv, kept_idx, k1, B, static_cast<uint4*>(y_kept));
 }
 
 cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
-                          void* y_kept, int num_sms, cudaStream_t stream) {
+                          void* y_kept, int num_sms, cudaStream_t stream, bool pdl) {
   const int Cv = C / 8;
   const int k1 = keep_k + 1;
-  const int rows = B * k1;
-  int blocks = (rows + 7) / 8;
+  int blocks = (B * k1 + 7) / 8;
   if (blocks > num_sms * 8) blocks = num_sms * 8;
-  const auto* yp = static_cast<const uint4*>(y);
-  auto* op = static_cast<uint4*>(y_kept);
+  const int vpl = (Cv + 31) / 32;
+  if (vpl <= 1) return launch_gather_t<1>(y, B, L, Cv, kept_idx, k1, y_kept, blocks, stream, pdl);
+  if (vpl <= 2) return launch_gather_t<2>(y, B, L, Cv, kept_idx, k1, y_kept, blocks, stream, pdl);
+  if (vpl <= 4) return launch_gather_t<4>(y, B, L, Cv, kept_idx, k1, y_kept, blocks, stream, pdl);
+  return launch_gather_t<8>(y, B, L, Cv, kept_idx, k1, y_kept, blocks, stream, pdl);
+}
+
+template <int VPL>
+static cudaError_t launch_sg_t(const float* partials, int NP, int L, int k, const void* y, int Cv,
+                               int B, int S, float* scores, int32_t* kept, void* y_kept,
+                               cudaStream_t stream, bool pdl) {
+  auto kern = select_gather_kernel<VPL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L - 1)));
+  if (e != cudaSuccess) return e;
+  return launch(kern, B * S, kSelGatherThreads, select_smem(L, k), stream, pdl, partials, NP, L, k,
+                static_cast<const uint4*>(y), Cv, S, scores, kept, static_cast<uint4*>(y_kept));
+}
+
+cudaError_t launch_select_gather(const float* partials, int num_partials, const void* y, int B,
+                                 int L, int C, int keep_k, float* scores, int32_t* kept_idx,
+                                 void* y_kept, int num_sms, cudaStream_t stream, bool pdl) {
+  // CTAs per sample: about one CTA per SM when B is small, one per sample otherwise
+  const int k1 = keep_k + 1;
+  int S = num_sms / B;
+  if (S > k1) S = k1;
+  if (S < 1) S = 1;
+  const int Cv = C / 8;
   const int vpl = (Cv + 31) / 32;
   if (vpl <= 1)
-    gather_kernel<1><<<blocks, 256, 0, stream>>>(yp, L, Cv, kept_idx, k1, rows, op);
-  else if (vpl <= 2)
-    gather_kernel<2><<<blocks, 256, 0, stream>>>(yp, L, Cv, kept_idx, k1, rows, op);
-  else if (vpl <= 4)
-    gather_kernel<4><<<blocks, 256, 0, stream>>>(yp, L, Cv, kept_idx, k1, rows, op);
-  else
-    gather_kernel<8><<<blocks, 256, 0, stream>>>(yp, L, Cv, kept_idx, k1, rows, op);
-  return cudaGetLastError();
+    return launch_sg_t<1>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
+                          stream, pdl);
+  if (vpl <= 2)
+    return launch_sg_t<2>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
+                          stream, pdl);
+  if (vpl <= 4)
+    return launch_sg_t<4>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
+                          stream, pdl);
+  return launch_sg_t<8>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
+                        stream, pdl);
 }
 
 }  // namespace rs

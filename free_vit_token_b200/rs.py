@@ -32,11 +32,14 @@ SIGNATURES = {
     "rs_ln_fc1_gelu": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_ln_fc1_gelu_staged": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_gelu_apply": (_i, [_fp, _fp, _i, _vp]),
+    "rs_ln_fold": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp, _fp, _fp, _vp]),
+    "rs_fc1_gelu_folded": (_i, [_vp, _fp, _vp, _fp, _fp, _i, _i, _i, _vp, _vp]),
     "rs_ln_fc1_gelu_noalloc": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_num_partials": (_i, [_i]),
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
+    "rs_select_gather": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
     "rs_status_string": (ctypes.c_char_p, [_i]),
     "rs_get_last_device_error": (_i, [_vp]),
     "rs_release_workspace": (None, []),
@@ -134,6 +137,35 @@ def rs_ln_fc1_gelu(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: Optional[torc
     return hidden
 
 
+def rs_ln_fold(W1: torch.Tensor, b1, gamma, beta, Wg: Optional[torch.Tensor] = None,
+               colG: Optional[torch.Tensor] = None, colC: Optional[torch.Tensor] = None,
+               stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    H, C = W1.shape
+    dev = W1.device
+    if Wg is None:
+        Wg = torch.empty(H, C, dtype=torch.bfloat16, device=dev)
+    if colG is None:
+        colG = torch.empty(H, dtype=torch.float32, device=dev)
+    if colC is None:
+        colC = torch.empty(H, dtype=torch.float32, device=dev)
+    st = lib().rs_ln_fold(_ptr(W1), _ptr(b1), _ptr(gamma), _ptr(beta), C, H, _ptr(Wg), _ptr(colG),
+                          _ptr(colC), _stream(stream))
+    _check(st, "rs_ln_fold")
+    return Wg, colG, colC
+
+
+def rs_fc1_gelu_folded(x2d: torch.Tensor, stats, Wg, colG, colC,
+                       hidden: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, C = x2d.shape
+    H = Wg.shape[0]
+    if hidden is None:
+        hidden = torch.empty(M, H, dtype=torch.bfloat16, device=x2d.device)
+    st = lib().rs_fc1_gelu_folded(_ptr(x2d), _ptr(stats), _ptr(Wg), _ptr(colG), _ptr(colC), M, C, H,
+                                  _ptr(hidden), _stream(stream))
+    _check(st, "rs_fc1_gelu_folded")
+    return hidden
+
+
 def rs_ln_fc1_gelu_staged(x2d: torch.Tensor, W1, b1, gamma, beta,
                           hidden: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     M, C = x2d.shape
@@ -197,6 +229,26 @@ def rs_select_topk(partials: torch.Tensor, B: int, L: int, keep_k: int,
                               _stream(stream))
     _check(st, "rs_select_topk")
     return scores, kept_idx
+
+
+def rs_select_gather(partials: torch.Tensor, y: torch.Tensor, keep_k: int,
+                     scores: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
+                     y_kept: Optional[torch.Tensor] = None, stream=None
+                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """partials [B*L, P] fp32, y [B, L, C] bf16 -> (scores, kept_idx, y_kept)."""
+    B, L, C = y.shape
+    P = partials.shape[-1]
+    dev = y.device
+    if scores is None:
+        scores = torch.empty(B, L, dtype=torch.float32, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
+    if y_kept is None:
+        y_kept = torch.empty(B, keep_k + 1, C, dtype=y.dtype, device=dev)
+    st = lib().rs_select_gather(_ptr(partials), P, _ptr(y), B, L, C, int(keep_k), _ptr(scores),
+                                _ptr(kept_idx), _ptr(y_kept), _stream(stream))
+    _check(st, "rs_select_gather")
+    return scores, kept_idx, y_kept
 
 
 def rs_gather_rows(y: torch.Tensor, kept_idx: torch.Tensor, keep_k: int,

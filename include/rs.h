@@ -104,6 +104,17 @@ int rs_ln_stats(const void* x, int M, int C, float* stats, void* stream);
 int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
                    const void* gamma, const void* beta, void* hidden, void* stream);
 
+/* The two launches that rs_ln_fc1_gelu makes after rs_ln_stats, exported on
+ * their own. rs_ln_fold: Wg [H, C] bf16, colG [H] and colC [H] fp32 as above
+ * (the fold of the LayerNorm's gamma, beta into fc1; W1 [H, C], b1 [H],
+ * gamma [C], beta [C] bf16). rs_fc1_gelu_folded: the tcgen05 GEMM with the
+ * folded-LN + GELU epilogue; stats [M, 2] from rs_ln_stats (8-byte aligned),
+ * colG and colC 16-byte aligned; hidden [M, H] bf16 output. */
+int rs_ln_fold(const void* W1, const void* b1, const void* gamma, const void* beta, int C, int H,
+               void* Wg, float* colG, float* colC, void* stream);
+int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const float* colG,
+                       const float* colC, int M, int C, int H, void* hidden, void* stream);
+
 /* The same result with the LayerNorm applied while staging fc1's A operand:
  * LN warps normalise each x' tile in shared memory (fp32 math, bf16 out)
  * before the tensor cores read it. Same arguments and workspace use. */
@@ -134,6 +145,13 @@ int rs_num_partials(int C);
  * partials [B*L, P] fp32 with 1 <= P <= 64; scores [B, L]; kept_idx [B, 1+keep_k]. */
 int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
                    float* scores, int32_t* kept_idx, void* stream);
+
+/* rs_select_topk followed by rs_gather_rows (same outputs), as rs_block_forward
+ * runs them: for L <= 256 one fused kernel in which every CTA ranks its
+ * sample's scores and copies a share of its kept rows. partials [B*L, P] fp32
+ * (1 <= P <= 64), y [B, L, C] bf16; outputs as for the two calls. */
+int rs_select_gather(const float* partials, int num_partials, const void* y, int B, int L, int C,
+                     int keep_k, float* scores, int32_t* kept_idx, void* y_kept, void* stream);
 
 /* Row gather, the pruned set x-tilde (§3.1):
  * y_kept[b, j, :] = y[b, kept_idx[b, j], :]. y [B, L, C] bf16; kept_idx

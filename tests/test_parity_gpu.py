@@ -27,7 +27,7 @@ def _device_ok():
 
 
 # --------------------------------------------------------------------------- select
-@pytest.mark.parametrize("L", [1, 2, 3, 197, 1098, 1569, 4100])
+@pytest.mark.parametrize("L", [1, 2, 3, 197, 256, 257, 1098, 1569, 4100])
 @pytest.mark.parametrize("ties", [False, True])
 def test_select_bitexact(L, ties):
     """fp32 score finalisation and top-k: bit-exact against the oracle's selection of
@@ -71,6 +71,23 @@ def test_gather_exact(C):
     out = rs.rs_gather_rows(y.to(dev), kept.to(dev), k)
     ref = np.stack([oracle.gather(y[b].float().numpy(), kept[b].numpy()) for b in range(B)])
     assert np.array_equal(out.float().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("L,C,k", [(197, 384, 137), (197, 768, 118), (256, 192, 0), (1, 64, 0),
+                                   (50, 2048, 49), (1569, 768, 784)])
+def test_select_gather_equals_separate_steps(L, C, k):
+    """rs_select_gather (fused for L <= 256) gives the bits of rs_select_topk +
+    rs_gather_rows."""
+    rs = _rs()
+    B = 7
+    parts = random_partials(B, L, 4, seed=L + C, ties=(L % 2 == 0)).to(dev)
+    g = torch.Generator().manual_seed(k + 1)
+    y = torch.randn(B, L, C, generator=g).to(torch.bfloat16).to(dev)
+    s1, k1 = rs.rs_select_topk(parts, B, L, k)
+    yk1 = rs.rs_gather_rows(y, k1, k)
+    s2, k2, yk2 = rs.rs_select_gather(parts, y, k)
+    torch.cuda.synchronize()
+    assert torch.equal(s1, s2) and torch.equal(k1, k2) and torch.equal(yk1, yk2)
 
 
 # --------------------------------------------------------------------------- LN stats
@@ -120,6 +137,29 @@ def test_fc1_hidden(M, C, H, variant):
                                 w64["W1"], w64["b1"]))
     parity.check_y(parity.f64(hid), ref, "hidden")
     _device_ok()
+
+
+def test_fc1_split_steps_equal_combined_step():
+    """rs_ln_stats + rs_ln_fold + rs_fc1_gelu_folded launch the same kernels as
+    rs_ln_fc1_gelu: identical bits."""
+    rs = _rs()
+    M, C, H = 333, 384, 1536
+    inp = random_block(1, M, C, H, seed=9, fg_rows=30)
+    x = inp.x.reshape(M, C).to(dev)
+    w = inp.weights[0]
+    W1, b1, g, be = (t.to(dev) for t in (w.W1, w.b1, w.gamma, w.beta))
+    ref = rs.rs_ln_fc1_gelu(x, W1, b1, g, be)
+    stats = rs.rs_ln_stats(x)
+    Wg, cg, cc = rs.rs_ln_fold(W1, b1, g, be)
+    hid = rs.rs_fc1_gelu_folded(x, stats, Wg, cg, cc)
+    torch.cuda.synchronize()
+    assert torch.equal(hid, ref)
+    # the fold itself: Wg = bf16(W1 * gamma), G = sum_c Wg, cb = W1 beta + b1
+    Wg_ref = (w.W1.float() * w.gamma.float()).to(torch.bfloat16)
+    assert torch.equal(Wg.cpu(), Wg_ref)
+    assert np.allclose(cg.cpu().double().numpy(), Wg_ref.double().sum(1).numpy(), rtol=1e-5, atol=1e-5)
+    cb_ref = parity.f64(w.W1) @ parity.f64(w.beta) + parity.f64(w.b1)
+    assert np.allclose(cc.cpu().double().numpy(), cb_ref, rtol=1e-4, atol=1e-5)
 
 
 def test_fc1_large_mean_rows():
