@@ -52,7 +52,8 @@ WsLayout ws_layout(int64_t M, int C, int H) {
   w.y = off;
   off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
   w.partials = off;
-  off = align_up(off + static_cast<size_t>(M) * (2 * C / rs::fc2_block_n(C)) * 4, 1024);
+  off = align_up(off + static_cast<size_t>(M) * (rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C)) * 4,
+                 1024);
   w.total = off;
   return w;
 }
@@ -106,8 +107,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Row-major bf16 [rows, inner] viewed as tiles of {box_inner elements, box_rows
-// rows}: 64-wide boxes use the 128-byte swizzle (GEMM operands), 32-wide boxes
-// the 64-byte swizzle (epilogue output boxes). Rows past the end read as zero
+// rows}: 64-wide boxes use the 128-byte swizzle (GEMM operands), 16-wide boxes
+// the 32-byte swizzle (epilogue output boxes). Rows past the end read as zero
 // and are not written.
 int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
               uint32_t box_inner = 64) {
@@ -117,8 +118,9 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   cuuint64_t strides[1] = {inner * 2};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw =
-      box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle sw = box_inner == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -193,7 +195,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, wB, C, H, bn));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, st.num_sms, s, /*pdl=*/true));
   return RS_OK;
 }
@@ -204,7 +206,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   CUtensorMap tmH, tmW, tmY;
   RS_TRY(make_tmap(&tmH, hidden, H, M, 128));
   RS_TRY(make_tmap(&tmW, W2, H, C, bn));
-  RS_TRY(make_tmap(&tmY, y, C, M, 32, 32));
+  RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   rs::MlpParams p{};
   p.M = M;
   p.N = C;
@@ -215,7 +217,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.out = static_cast<__nv_bfloat16*>(y);
   p.resid = static_cast<const __nv_bfloat16*>(x);
   p.partials = partials;
-  p.num_partials = 2 * p.n_blocks;
+  p.num_partials = rs::kFc2PartialsPerTile * p.n_blocks;
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, st.num_sms, s, pdl));
@@ -240,7 +242,9 @@ const char* rs_status_string(int status) {
   }
 }
 
-int rs_num_partials(int C) { return check_width(C) == RS_OK ? 2 * C / rs::fc2_block_n(C) : 0; }
+int rs_num_partials(int C) {
+  return check_width(C) == RS_OK ? rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C) : 0;
+}
 
 uint64_t rs_workspace_bytes(int B, int L, int C, int H) {
   if (B < 0 || L < 1 || check_width(C) != RS_OK || check_hidden(H) != RS_OK) return 0;
@@ -328,7 +332,7 @@ int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const 
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, Wg, C, H, bn));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, 32, 32));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
@@ -456,7 +460,7 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
   void* hidden = ws + w.hidden;
   void* y = ws + w.y;
   float* partials = reinterpret_cast<float*>(ws + w.partials);
-  const int np = 2 * C / rs::fc2_block_n(C);
+  const int np = rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
 
   RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
   RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s, /*pdl=*/true));

@@ -17,6 +17,14 @@ constexpr int kEpiGelu = 0;              // fc1 epilogue: + b1, erf-GELU, bf16 s
 constexpr int kEpiResidShift = 1;        // fc2 epilogue: + b2, residual, shift partials
 constexpr int kEpiGeluFold = 2;          // fc1 epilogue: folded LN (mean, rstd, G, cb), erf-GELU
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // one pipeline wait: 4 s
+// The GEMM epilogue writes its outputs (hidden, y) through per-warp boxes of
+// 32 rows x 16 bf16 columns with the 32-byte swizzle; output tensor maps use
+// this box.
+constexpr int kEpiBoxRows = 32;
+constexpr int kEpiBoxCols = 16;
+// fc2 writes this many shift partials per row and 128 x BN output tile (one per
+// epilogue column group).
+constexpr int kFc2PartialsPerTile = 2;
 
 // Launches `kern` on `stream`; with `pdl` the launch may begin while the
 // previous kernel in the stream is still running (every kernel of this library

@@ -32,12 +32,12 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;                         // one 128-byte swizzle row of bf16
 constexpr int kAStageBytes = kBM * kBK * 2;     // 16 KB
 constexpr int kEpiWarp0 = 4;
-constexpr int kNumEpiWarps = 8;
-constexpr int kLnWarp0 = 12;
+constexpr int kMaxEpiWarps = 16;
+constexpr int kLnWarp0 = 12;  // staged-LN kernel: after its 8 epilogue warps
 constexpr int kNumLnWarps = 4;
 constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 constexpr int kCtrlBytes = 512;                 // barriers, TMEM slot, abort flag
-constexpr int kEpiBoxBytes = 32 * 32 * 2;       // one warp's 32 x 32 bf16 output box
+constexpr int kEpiBoxBytes = kEpiBoxRows * kEpiBoxCols * 2;  // one warp's output box
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kVecMaxBytes = 2 * 256 * 4;       // one tile's column vectors (fold: G and cb)
@@ -54,7 +54,7 @@ __host__ __device__ constexpr int vec_stride(int bn, int epi) {
 __host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
   // alignment slack + control block + gamma/beta (bf16, up to RS_MAX_C each) +
   // the epilogue's per-warp output boxes + two tiles' column vectors
-  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + kNumEpiWarps * kEpiBoxBytes +
+  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + kMaxEpiWarps * kEpiBoxBytes +
          2 * kVecMaxBytes;
 }
 __host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
@@ -62,11 +62,16 @@ __host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
              ? 6
              : (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn);
 }
-__host__ __device__ constexpr int num_threads(bool ln) { return (ln ? 16 : 12) * 32; }
+// Epilogue warps EW: 8 (two per TMEM lane quadrant) or 16 (four). 16 pays off
+// only where the epilogue's arithmetic rivals a short main loop (fc1 with
+// C <= 512); the staged-LN kernel always uses 8 (its LN warps need registers).
+__host__ __device__ constexpr int num_threads(bool ln, int ew) {
+  return (kEpiWarp0 + ew + (ln ? kNumLnWarps : 0)) * 32;
+}
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K) {
   return 1024 + static_cast<size_t>(num_stages(bn, ln, epi)) * stage_bytes(bn) +
-         kNumEpiWarps * kEpiBoxBytes + 2 * vec_stride(bn, epi) + kCtrlBytes +
+         kMaxEpiWarps * kEpiBoxBytes + 2 * vec_stride(bn, epi) + kCtrlBytes +
          (ln ? 4 * static_cast<size_t>(K) : 0);
 }
 
@@ -121,14 +126,17 @@ cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
-template <int BN, bool LN_A, int EPI>
-__global__ void __launch_bounds__(num_threads(LN_A), 1)
+template <int BN, bool LN_A, int EPI, int EW>
+__global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     mlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const MlpParams p) {
   constexpr int kBStageBytes = BN * kBK * 2;
   constexpr int STAGES = num_stages(BN, LN_A, EPI);
   constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN);
-  constexpr int kOutBytes = kNumEpiWarps * kEpiBoxBytes;
+  constexpr int kNumEpiWarps = EW;
+  static_assert(EW == 8 || EW == 16, "epilogue warps");
+  static_assert(!LN_A || EW == 8, "staged-LN kernel: 8 epilogue warps");
+  constexpr int kOutBytes = kMaxEpiWarps * kEpiBoxBytes;
   constexpr int kVecBytes = vec_bytes(BN, EPI);
   constexpr int kVecStride = vec_stride(BN, EPI);
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
@@ -288,17 +296,19 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
     __syncwarp();
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    // Warp -> TMEM lane quadrant q (rows 32q..32q+31 of the tile) and one half
-    // of the BN columns, in 32-column chunks: the TMEM load (and for fc2 the
-    // residual rows) of chunk n+1 are in flight while chunk n is processed. The
-    // accumulator goes back to the MMA warp as soon as its last chunk is in
-    // registers. Every chunk leaves through the warp's 32 x 32 output box
-    // (64-byte swizzle: 16-byte chunk j of row r at j ^ ((r >> 1) & 3)) and a
-    // TMA store; rows past M are clipped by the store.
+    // Warp -> TMEM lane quadrant q (rows 32q..32q+31 of the tile) and one of
+    // kNumEpiWarps/4 column groups of the BN columns, in 16-column chunks: the
+    // TMEM load (and for fc2 the residual row slice) of chunk n+1 is in flight
+    // while chunk n is processed. The accumulator goes back to the MMA warp as
+    // soon as its last chunk is in registers. Every chunk leaves through the
+    // warp's 32 x 16 output box (32-byte swizzle: 16-byte half j of row r at
+    // j ^ ((r >> 2) & 1)) and a TMA store; rows past M are clipped by the store.
+    constexpr int kGroups = kNumEpiWarps / 4;
+    constexpr int kCols = BN / kGroups;  // columns of one warp
+    constexpr int NCH = kCols / kEpiBoxCols;
+    static_assert(kCols % kEpiBoxCols == 0, "chunking");
     const int q = warp & 3;
-    const int half = (warp - kEpiWarp0) >> 2;
-    constexpr int kHalf = BN / 2;
-    constexpr int NCH = kHalf / 32;
+    const int grp = (warp - kEpiWarp0) >> 2;
     uint8_t* box = sOut + (warp - kEpiWarp0) * kEpiBoxBytes;
     const uint32_t box_u32 = smem_u32(box);
     int acc = 0;
@@ -318,8 +328,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
       const int row = m_blk * kBM + q * 32 + lane;
       const bool row_ok = row < p.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN + half * kHalf);
-      const int col0 = n_blk * BN + half * kHalf;
+                             static_cast<uint32_t>(acc * BN + grp * kCols);
+      const int col0 = n_blk * BN + grp * kCols;
       const uint32_t vec_u32 = smem_u32(sVec + acc * kVecStride);
       float part = 0.f;
       uint64_t nmu2 = 0, rs2 = 0;  // folded LN: (-mean, -mean), (rstd, rstd) of this row
@@ -329,30 +339,31 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         nmu2 = f2pack(-st.x, -st.x);
         rs2 = f2pack(st.y, st.y);
       }
-      const uint4* xrow = reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.N + col0);
-      uint32_t ra[32], rb[32];
-      uint4 xa[4] = {}, xb[4] = {};
-      tmem_ld32_async(t_row, ra);
+      const uint4* xrow =
+          reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.N + col0);
+      uint32_t ra[16], rb[16];
+      uint4 xa[2] = {}, xb[2] = {};
+      tmem_ld16_async(t_row, ra);
       if constexpr (EPI == kEpiResidShift) {
         if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) xa[v] = __ldg(xrow + v);
+          xa[0] = __ldg(xrow);
+          xa[1] = __ldg(xrow + 1);
         }
       }
 #pragma unroll
       for (int n = 0; n < NCH; ++n) {
-        uint32_t(&r)[32] = (n & 1) ? rb : ra;
-        uint32_t(&nx)[32] = (n & 1) ? ra : rb;
-        uint4(&xv)[4] = (n & 1) ? xb : xa;
-        uint4(&xn)[4] = (n & 1) ? xa : xb;
+        uint32_t(&r)[16] = (n & 1) ? rb : ra;
+        uint32_t(&nx)[16] = (n & 1) ? ra : rb;
+        uint4(&xv)[2] = (n & 1) ? xb : xa;
+        uint4(&xn)[2] = (n & 1) ? xa : xb;
         tmem_wait_ld();
-        reg_fence(r);
+        reg_fence16(r);
         if (n + 1 < NCH) {
-          tmem_ld32_async(t_row + (n + 1) * 32, nx);
+          tmem_ld16_async(t_row + (n + 1) * 16, nx);
           if constexpr (EPI == kEpiResidShift) {
             if (row_ok) {
-#pragma unroll
-              for (int v = 0; v < 4; ++v) xn[v] = __ldg(xrow + (n + 1) * 4 + v);
+              xn[0] = __ldg(xrow + (n + 1) * 2);
+              xn[1] = __ldg(xrow + (n + 1) * 2 + 1);
             }
           }
         } else {
@@ -360,13 +371,13 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        const int c = n * 32;
-        const uint32_t cvec = (half * kHalf + c);  // column of this chunk within the tile
-        uint32_t outw[16];
+        const int c = n * 16;
+        const uint32_t cvec = grp * kCols + c;  // column of this chunk within the tile
+        uint32_t outw[8];
         if constexpr (EPI == kEpiGeluFold) {
           // z = rstd * (acc - mean * G[col]) + cb[col], two columns per step
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < 4; ++v) {
             const uint4 g4 = lds128(vec_u32 + (cvec + 4 * v) * 4);
             const uint4 c4 = lds128(vec_u32 + BN * 4 + (cvec + 4 * v) * 4);
             const uint64_t ga = (static_cast<uint64_t>(g4.y) << 32) | g4.x;
@@ -385,9 +396,9 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
             outw[2 * v + 1] = pack_bf16x2(g1.x, g1.y);
           }
         } else {
-          uint32_t bw[16];
+          uint32_t bw[8];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 2; ++v) {
             const uint4 b4 = lds128(vec_u32 + (cvec + 8 * v) * 2);
             bw[4 * v] = b4.x;
             bw[4 * v + 1] = b4.y;
@@ -396,7 +407,7 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
           }
           if constexpr (EPI == kEpiGelu) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 8; ++e) {
               const float2 g = f2unpack(gelu2(f2pack(__uint_as_float(r[2 * e]) + bf16lo(bw[e]),
                                                      __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]))));
               outw[e] = pack_bf16x2(g.x, g.y);
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
           } else {
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 8; ++e) {
               const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
               const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
               const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
@@ -422,10 +433,11 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         }
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          sts128(box_u32 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
-                 make_uint4(outw[4 * j], outw[4 * j + 1], outw[4 * j + 2], outw[4 * j + 3]));
+        const uint32_t sw = (lane >> 2) & 1;
+        sts128(box_u32 + lane * 32 + ((0u ^ sw) << 4),
+               make_uint4(outw[0], outw[1], outw[2], outw[3]));
+        sts128(box_u32 + lane * 32 + ((1u ^ sw) << 4),
+               make_uint4(outw[4], outw[5], outw[6], outw[7]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -434,7 +446,8 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
         }
       }
       if constexpr (EPI == kEpiResidShift) {
-        if (row_ok) p.partials[static_cast<size_t>(row) * p.num_partials + n_blk * 2 + half] = part;
+        if (row_ok)
+          p.partials[static_cast<size_t>(row) * p.num_partials + n_blk * kGroups + grp] = part;
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
@@ -520,17 +533,17 @@ __global__ void __launch_bounds__(num_threads(LN_A), 1)
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int BN, bool LN_A, int EPI>
+template <int BN, bool LN_A, int EPI, int EW = 8>
 static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                const CUtensorMap& tmOut, const MlpParams& p, int num_sms,
                                cudaStream_t stream, bool pdl) {
-  auto kern = mlp_gemm_kernel<BN, LN_A, EPI>;
+  auto kern = mlp_gemm_kernel<BN, LN_A, EPI, EW>;
   const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  return launch(kern, grid, num_threads(LN_A), smem, stream, pdl, tmA, tmB, tmOut, p);
+  return launch(kern, grid, num_threads(LN_A, EW), smem, stream, pdl, tmA, tmB, tmOut, p);
 }
 
 int fc1_block_n(int H) { return H % 256 == 0 ? 256 : (H % 128 == 0 ? 128 : 64); }
@@ -546,6 +559,13 @@ cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CU
       case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
       case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
       default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+    }
+  }
+  if (p.K <= 512) {
+    switch (bn) {
+      case 256: return launch_gemm<256, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+      case 128: return launch_gemm<128, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+      default: return launch_gemm<64, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
     }
   }
   switch (bn) {

@@ -70,8 +70,9 @@ int encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
   cuuint64_t strides[1] = {inner * 2};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw =
-      box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle sw = box_inner == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
@@ -119,7 +120,7 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
   const int bn = rs::fc1_block_n(H);
   CUtensorMap tmX, tmW, tmHid;
   if (encode_map(&tmX, x, C, M, 128, 64) != RS_OK || encode_map(&tmW, wg, C, H, bn, 64) != RS_OK ||
-      encode_map(&tmHid, hidden, H, M, 32, 32) != RS_OK)
+      encode_map(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols) != RS_OK)
     return RS_ERR_CUDA;
   rs::MlpParams p{};
   p.M = M;

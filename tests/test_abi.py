@@ -35,7 +35,7 @@ def test_status_strings():
 
 
 def test_num_partials_and_workspace():
-    assert rs.rs_num_partials(384) == 4      # two 192-wide column groups, two halves each
+    assert rs.rs_num_partials(384) == 4      # two 192-wide tiles, two column groups each
     assert rs.rs_num_partials(768) == 6
     assert rs.rs_num_partials(1024) == 8
     assert rs.rs_num_partials(192) == 2
