@@ -108,21 +108,68 @@ __device__ __forceinline__ uint64_t gelu2(uint64_t z2) {
   return fmul2(z2, f2pack(__saturatef(fmaf(zf.x, pf.x, 0.5f)), __saturatef(fmaf(zf.y, pf.y, 0.5f))));
 }
 
-// Elementwise GELU with the same arithmetic as the fc1 epilogue.
+// Near-range GELU of two lanes, valid for |z| <= RS_GELU_NEAR_Z, given
+// u = RS_GELU_NEAR_K z^2 - 1 (in [-1, 1] there): Phi = 1/2 + z P(u), degree 8,
+// no clamp and no saturation (max |error| 5.6e-7).
+__device__ __forceinline__ uint64_t gelu2_near(uint64_t z2, uint64_t u2) {
+  uint64_t p = kpair(RS_GELU_NEAR_P8);
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P7));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P6));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P5));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P4));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P3));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P2));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P1));
+  p = ffma2(p, u2, kpair(RS_GELU_NEAR_P0));
+  return fmul2(z2, ffma2(z2, p, kpair(0.5f)));
+}
+
+// GELU of N lane pairs held by a warp: the near-range polynomial when every
+// value the warp holds has |z| <= RS_GELU_NEAR_Z (a warp-uniform choice), the
+// full-range one otherwise. Every lane of the warp must call it.
+template <int N>
+__device__ __forceinline__ void gelu2_block(const uint64_t (&z2)[N], uint64_t (&g2)[N]) {
+  uint64_t u2[N];
+  float um = -1.f;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    u2[i] = ffma2(fmul2(z2[i], kpair(RS_GELU_NEAR_K)), z2[i], kpair(-1.f));
+    const float2 uf = f2unpack(u2[i]);
+    um = fmaxf(um, fmaxf(uf.x, uf.y));
+  }
+  if (__all_sync(0xffffffffu, um <= 1.f)) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) g2[i] = gelu2_near(z2[i], u2[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) g2[i] = gelu2(z2[i]);
+  }
+}
+
+// Elementwise GELU with the same arithmetic as the fc1 epilogue (grid-stride,
+// every lane of a warp stays active for the warp-uniform range choice).
 __global__ void gelu_apply_kernel(const float* __restrict__ z, float* __restrict__ out, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 g = f2unpack(gelu2(f2pack(z[i], z[i + 1])));
-    out[i] = g.x;
-    out[i + 1] = g.y;
-  } else if (i < n) {
-    out[i] = f2unpack(gelu2(f2pack(z[i], 0.f))).x;
+  const int pairs = (n + 1) / 2;
+  const int stride = gridDim.x * blockDim.x;
+  const int iters = (pairs + stride - 1) / stride;
+  for (int it = 0; it < iters; ++it) {
+    const int pi = it * stride + blockIdx.x * blockDim.x + threadIdx.x;
+    const int i = 2 * pi;
+    const float z0 = i < n ? z[i] : 0.f;
+    const float z1 = i + 1 < n ? z[i + 1] : 0.f;
+    uint64_t zz[1] = {f2pack(z0, z1)}, gg[1];
+    gelu2_block<1>(zz, gg);
+    const float2 g = f2unpack(gg[0]);
+    if (i < n) out[i] = g.x;
+    if (i + 1 < n) out[i + 1] = g.y;
   }
 }
 
 cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream) {
   const int pairs = (n + 1) / 2;
-  gelu_apply_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(z, out, n);
+  int blocks = (pairs + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  gelu_apply_kernel<<<blocks, 256, 0, stream>>>(z, out, n);
   return cudaGetLastError();
 }
 
@@ -376,6 +423,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         uint32_t outw[8];
         if constexpr (EPI == kEpiGeluFold) {
           // z = rstd * (acc - mean * G[col]) + cb[col], two columns per step
+          uint64_t z2[8], g2[8];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             const uint4 g4 = lds128(vec_u32 + (cvec + 4 * v) * 4);
@@ -384,16 +432,19 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
             const uint64_t gb = (static_cast<uint64_t>(g4.w) << 32) | g4.z;
             const uint64_t ca = (static_cast<uint64_t>(c4.y) << 32) | c4.x;
             const uint64_t cb = (static_cast<uint64_t>(c4.w) << 32) | c4.z;
-            const uint64_t za = ffma2(
+            z2[2 * v] = ffma2(
                 rs2, ffma2(nmu2, ga, f2pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]))),
                 ca);
-            const uint64_t zb = ffma2(
+            z2[2 * v + 1] = ffma2(
                 rs2,
                 ffma2(nmu2, gb, f2pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]))),
                 cb);
-            const float2 g0 = f2unpack(gelu2(za)), g1 = f2unpack(gelu2(zb));
-            outw[2 * v] = pack_bf16x2(g0.x, g0.y);
-            outw[2 * v + 1] = pack_bf16x2(g1.x, g1.y);
+          }
+          gelu2_block<8>(z2, g2);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 g = f2unpack(g2[e]);
+            outw[e] = pack_bf16x2(g.x, g.y);
           }
         } else {
           uint32_t bw[8];
@@ -406,10 +457,15 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
             bw[4 * v + 3] = b4.w;
           }
           if constexpr (EPI == kEpiGelu) {
+            uint64_t z2[8], g2[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              z2[e] = f2pack(__uint_as_float(r[2 * e]) + bf16lo(bw[e]),
+                             __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]));
+            gelu2_block<8>(z2, g2);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float2 g = f2unpack(gelu2(f2pack(__uint_as_float(r[2 * e]) + bf16lo(bw[e]),
-                                                     __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]))));
+              const float2 g = f2unpack(g2[e]);
               outw[e] = pack_bf16x2(g.x, g.y);
             }
           } else {

@@ -106,11 +106,16 @@ def test_ln_stats(C):
 
 # --------------------------------------------------------------------------- GELU
 def test_gelu_apply_error_bound():
-    """The epilogue's GELU against the exact z * Phi(z) (fp64 oracle) on a dense grid:
-    |error| <= 1.5e-6 everywhere and <= 3e-7 * max(1, |z|) relative to scale."""
+    """The epilogue's GELU against the exact z * Phi(z) (fp64 oracle): |error| <= 1.5e-6,
+    on warps whose values all lie in |z| <= 3 (the near-range polynomial) and on warps
+    holding wider values (the full-range one)."""
     rs = _rs()
-    z = torch.cat([torch.linspace(-12, 12, 400001), torch.randn(100000) * 3,
-                   torch.tensor([0.0, -0.0, 1e-30, -1e-30, 5.3, -5.3, 40.0, -40.0])]).float()
+    g = torch.Generator().manual_seed(2)
+    z = torch.cat([torch.linspace(-3, 3, 262144),                 # whole warps in range
+                   torch.linspace(-12, 12, 400001),               # mixed warps
+                   torch.randn(100000, generator=g) * 0.4,        # hidden-like values
+                   torch.tensor([0.0, -0.0, 1e-30, -1e-30, 3.0, -3.0, 5.3, -5.3, 40.0, -40.0])]
+                  ).float()
     g = rs.rs_gelu_apply(z.to(dev)).cpu().double().numpy()
     ref = oracle.gelu(z.double().numpy())
     err = np.abs(g - ref)
