@@ -56,6 +56,39 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+# ----------------------------------------------------------------------------- ncu traffic
+GEMM_SOURCES = ["free_vit_token_b200/csrc/rs_mlp.cu", "free_vit_token_b200/csrc/rs_ptx.cuh",
+                "free_vit_token_b200/csrc/rs_gelu_poly.h", "free_vit_token_b200/csrc/rs_internal.h"]
+
+
+def gemm_source_hash() -> str:
+    """Digest of the GEMM kernels' sources: DRAM traffic measured by ncu is reported
+    only while the kernels are the ones that were profiled."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from
+    profiles/traffic.json, or None when absent or taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    want = gemm_source_hash()
+    for e in d.get("entries", []):
+        if e.get("kernel") == kernel and e.get("workload") == workload and \
+                e.get("source_hash") == want:
+            return float(e["dram_bytes_per_launch"])
+    return None
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -120,29 +153,8 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- dist
-def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-
-
-def max_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+from free_vit_token_b200.replicas import (barrier, env_ranks, init as dist_init,  # noqa: E402
+                                          job_throughput, max_over_ranks, rank_seed, shutdown)
 
 
 # ----------------------------------------------------------------------------- oracle leg
@@ -188,7 +200,8 @@ def main():
                     help="seconds of oracle work for the cpu_baseline leg (0 = skip)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
-    world, rank, local = dist_setup(args.gpus)
+    # the reference arm runs on rank 0 alone and joins no process group
+    world, rank, local = dist_init("nccl") if args.impl == "rs" else env_ranks()
     tokens_per_step = sum(wl.tokens(s) for s in range(wl.stages))
     config = {"workload": wl.name, "B": wl.B, "L": wl.L, "C": wl.C, "H": wl.H,
               "keep_k": list(wl.keep_k), "stages": wl.stages,
@@ -225,7 +238,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    inp = make_inputs(wl, seed=rank)
+    inp = make_inputs(wl, seed=rank_seed(0, rank))
     x = inp.x.to(dev)
     W = [[t.to(dev) for t in (w.W1, w.b1, w.W2, w.b2, w.gamma, w.beta)] for w in inp.weights]
     stream = torch.cuda.current_stream(dev)
@@ -234,7 +247,7 @@ def main():
              torch.empty(wl.B, wl.stage_L(s), dtype=torch.float32, device=dev))
             for s, k in enumerate(wl.keep_k)]
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def l2_flush():
         flush_w.zero_()
@@ -267,11 +280,11 @@ def main():
     barrier(world)
     clocks.mark_end = time.time()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), world)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     status = rs.rs_get_last_device_error()
     assert status == 0, rs.status_string(status)
     ms_per_step = total_ms / args.steps
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(tokens_per_step, args.steps, total_ms, world)
 
     # ---- per-kernel breakdown (the same kernels, one step-level entry point each)
     names = ("stats", "fold", "fc1", "fc2", "select_gather")
@@ -353,8 +366,8 @@ def main():
         e2e_ev.append((a, b))
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world) / n_e2e
-    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev) / n_e2e
+    e2e_value = job_throughput(tokens_per_step, 1, e2e_ms, world)
     clocks.stop()
 
     cpu = None
@@ -372,7 +385,8 @@ def main():
         "config": config,
         "roofline": {"bound": "tensor", "kernel": f"{dominant} (tcgen05 GEMM)",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": achieved_tf / peak_tf, "traffic": None,
+                     "frac": achieved_tf / peak_tf,
+                     "traffic": ncu_traffic(dominant, wl.name) if wl.stages == 1 else None,
                      "peak_source": f"{peaks['source']} bf16 burst",
                      "kernel_ms": fc_ms[dominant]},
         "block_tflops": block_flops / (ms_per_step / 1e3) / 1e12,
@@ -391,8 +405,7 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     rs.rs_release_workspace()
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    shutdown(world)
     return 0
 
 

@@ -8,6 +8,7 @@ from .rs import (  # noqa: F401
     lib,
     rs_block_forward,
     rs_fc2_residual_shift,
+    rs_debug_fc1_skip_load,
     rs_fc1_gelu_folded,
     rs_gather_rows,
     rs_gelu_apply,

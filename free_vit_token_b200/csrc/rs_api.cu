@@ -176,6 +176,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
+  p.debug_skip_kb = -1;
   const void* wB = W1;
   if (staged) {
     RS_CUDA(rs::launch_ln_stats(x, M, C, stats, st.num_sms, s));
@@ -220,6 +221,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.num_partials = rs::kFc2PartialsPerTile * p.n_blocks;
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
+  p.debug_skip_kb = -1;
   RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, st.num_sms, s, pdl));
   return RS_OK;
 }
@@ -345,8 +347,56 @@ int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const 
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = st->err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
+  p.debug_skip_kb = -1;
   RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, st->num_sms,
                          static_cast<cudaStream_t>(stream)));
+  return RS_OK;
+}
+
+int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                           const void* gamma, const void* beta, void* hidden, int skip_kblock,
+                           int timeout_us, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (M == 0) return RS_OK;
+  if (skip_kblock < 0 || skip_kblock >= C / 64 || timeout_us < 1 || timeout_us > 10000000)
+    return RS_ERR_SHAPE;
+  if (!x || !W1 || !b1 || !gamma || !beta || !hidden) return RS_ERR_NULL;
+  if (!al16(x) || !al16(W1) || !al16(b1) || !al16(gamma) || !al16(beta) || !al16(hidden))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  const WsLayout w = ws_layout(M, C, H);
+  RS_TRY(ensure_ws(*st, w.fc1_total));
+  uint8_t* ws = static_cast<uint8_t*>(st->ws);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* stats = reinterpret_cast<float*>(ws + w.stats);
+  void* wg = ws + w.wg;
+  float* colg = reinterpret_cast<float*>(ws + w.colg);
+  float* colc = reinterpret_cast<float*>(ws + w.colc);
+  RS_CUDA(rs::launch_ln_prep(x, M, C, stats, W1, gamma, beta, b1, H, wg, colg, colc, st->num_sms,
+                             s));
+  const int bn = rs::fc1_block_n(H);
+  CUtensorMap tmX, tmW, tmHid;
+  RS_TRY(make_tmap(&tmX, x, C, M, 128));
+  RS_TRY(make_tmap(&tmW, wg, C, H, bn));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
+  rs::MlpParams p{};
+  p.M = M;
+  p.N = H;
+  p.K = C;
+  p.n_blocks = H / bn;
+  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.stats = reinterpret_cast<const float2*>(stats);
+  p.colG = colg;
+  p.colC = colc;
+  p.out = static_cast<__nv_bfloat16*>(hidden);
+  p.err = st->err;
+  p.timeout_ns = static_cast<unsigned long long>(timeout_us) * 1000ull;
+  p.debug_skip_kb = skip_kblock;
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, st->num_sms, s));
   return RS_OK;
 }
 

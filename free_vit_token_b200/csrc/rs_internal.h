@@ -60,6 +60,8 @@ struct MlpParams {
   int num_partials;               // 2 * n_blocks (fc2)
   int* err;                       // device status flag
   unsigned long long timeout_ns;  // limit of one pipeline wait
+  int debug_skip_kb;              // test hook: CTA 0 skips this k-block's loads of its
+                                  // first tile (-1: off)
 };
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K);

@@ -286,12 +286,16 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], stage_bytes(BN));
-          tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, m_blk * kBM);
-          tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, n_blk * BN);
+          // test hook: leave one stage unfilled so the consumer's wait runs out
+          const bool skip = kb == p.debug_skip_kb && blockIdx.x == 0 && tile == blockIdx.x;
+          if (!skip) {
+            mbar_arrive_expect_tx(&full[stage], stage_bytes(BN));
+            tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, m_blk * kBM);
+            tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, n_blk * BN);
 #pragma unroll
-          for (int s = 0; s < STAGES; ++s)
-            if (s == stage) pend[s] = static_cast<int>(phase);
+            for (int s = 0; s < STAGES; ++s)
+              if (s == stage) pend[s] = static_cast<int>(phase);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;

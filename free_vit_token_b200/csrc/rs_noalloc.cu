@@ -134,6 +134,7 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
+  p.debug_skip_kb = -1;
   if (rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, num_sms, st) != cudaSuccess) {
     cudaGetLastError();
     return RS_ERR_CUDA;

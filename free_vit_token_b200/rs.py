@@ -32,6 +32,7 @@ SIGNATURES = {
     "rs_ln_fc1_gelu": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_ln_fc1_gelu_staged": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_gelu_apply": (_i, [_fp, _fp, _i, _vp]),
+    "rs_debug_fc1_skip_load": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp]),
     "rs_ln_fold": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp, _fp, _fp, _vp]),
     "rs_fc1_gelu_folded": (_i, [_vp, _fp, _vp, _fp, _fp, _i, _i, _i, _vp, _vp]),
     "rs_ln_fc1_gelu_noalloc": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -188,6 +189,17 @@ def rs_ln_fc1_gelu_noalloc(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: torch
                                       _ptr(beta), _ptr(hidden), _stream(stream))
     _check(st, "rs_ln_fc1_gelu_noalloc")
     return hidden
+
+
+def rs_debug_fc1_skip_load(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: torch.Tensor,
+                           skip_kblock: int, timeout_us: int, stream=None) -> None:
+    """Test hook: fc1 with one k-block load withheld (see include/rs.h)."""
+    M, C = x2d.shape
+    H = W1.shape[0]
+    st = lib().rs_debug_fc1_skip_load(_ptr(x2d), M, C, H, _ptr(W1), _ptr(b1), _ptr(gamma),
+                                      _ptr(beta), _ptr(hidden), int(skip_kblock), int(timeout_us),
+                                      _stream(stream))
+    _check(st, "rs_debug_fc1_skip_load")
 
 
 def rs_gelu_apply(z: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -183,6 +183,18 @@ int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, 
 int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const void* W1, const void* b1,
                            const void* gamma, const void* beta, void* hidden, void* stream);
 
+/* Test hook for failure detection (no counterpart in the paper): runs
+ * rs_ln_fc1_gelu except that CTA 0's producer leaves k-block `skip_kblock`
+ * (0 <= skip_kblock < C/64) of its first tile unloaded, so the MMA warp's wait
+ * on that stage cannot complete. Every pipeline wait is limited to `timeout_us`
+ * (1 .. 10^7). The kernel then records RS_ERR_DEVICE_TIMEOUT in the device
+ * flag, drains its own in-flight copies and MMAs, frees its tensor memory and
+ * returns; rs_get_last_device_error reports the status and the CUDA context
+ * stays usable. `hidden` is left partly unwritten. */
+int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                           const void* gamma, const void* beta, void* hidden, int skip_kblock,
+                           int timeout_us, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* rs_status_string(int status);
 
