@@ -166,12 +166,13 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
             bool staged, cudaStream_t s) {
   float* stats = reinterpret_cast<float*>(ws + w.stats);
   const int bn = rs::fc1_block_n(H);
+  const bool pair = rs::gemm_pair(M, C, staged);
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
   p.K = C;
   p.n_blocks = H / bn;
-  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.num_tiles = rs::gemm_num_tiles(M, p.n_blocks, pair);
   p.stats = reinterpret_cast<const float2*>(stats);
   p.out = static_cast<__nv_bfloat16*>(hidden);
   p.err = st.err;
@@ -195,25 +196,26 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   }
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
-  RS_TRY(make_tmap(&tmW, wB, C, H, bn));
+  RS_TRY(make_tmap(&tmW, wB, C, H, rs::gemm_b_box_rows(bn, pair)));
   RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
-  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, st.num_sms, s, /*pdl=*/true));
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, pair, st.num_sms, s, /*pdl=*/true));
   return RS_OK;
 }
 
 int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H, const void* W2,
             const void* b2, void* y, float* partials, cudaStream_t s, bool pdl = false) {
   const int bn = rs::fc2_block_n(C);
+  const bool pair = rs::gemm_pair(M, H, false);
   CUtensorMap tmH, tmW, tmY;
   RS_TRY(make_tmap(&tmH, hidden, H, M, 128));
-  RS_TRY(make_tmap(&tmW, W2, H, C, bn));
+  RS_TRY(make_tmap(&tmW, W2, H, C, rs::gemm_b_box_rows(bn, pair)));
   RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   rs::MlpParams p{};
   p.M = M;
   p.N = C;
   p.K = H;
   p.n_blocks = C / bn;
-  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.num_tiles = rs::gemm_num_tiles(M, p.n_blocks, pair);
   p.bias = static_cast<const __nv_bfloat16*>(b2);
   p.out = static_cast<__nv_bfloat16*>(y);
   p.resid = static_cast<const __nv_bfloat16*>(x);
@@ -222,7 +224,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
-  RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, st.num_sms, s, pdl));
+  RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, pair, st.num_sms, s, pdl));
   return RS_OK;
 }
 
@@ -331,16 +333,17 @@ int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const 
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
   const int bn = rs::fc1_block_n(H);
+  const bool pair = rs::gemm_pair(M, C, false);
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
-  RS_TRY(make_tmap(&tmW, Wg, C, H, bn));
+  RS_TRY(make_tmap(&tmW, Wg, C, H, rs::gemm_b_box_rows(bn, pair)));
   RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
   p.K = C;
   p.n_blocks = H / bn;
-  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.num_tiles = rs::gemm_num_tiles(M, p.n_blocks, pair);
   p.stats = reinterpret_cast<const float2*>(stats);
   p.colG = colG;
   p.colC = colC;
@@ -348,7 +351,7 @@ int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const 
   p.err = st->err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
-  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, st->num_sms,
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, pair, st->num_sms,
                          static_cast<cudaStream_t>(stream)));
   return RS_OK;
 }
@@ -379,16 +382,17 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   RS_CUDA(rs::launch_ln_prep(x, M, C, stats, W1, gamma, beta, b1, H, wg, colg, colc, st->num_sms,
                              s));
   const int bn = rs::fc1_block_n(H);
+  const bool pair = rs::gemm_pair(M, C, false);
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
-  RS_TRY(make_tmap(&tmW, wg, C, H, bn));
+  RS_TRY(make_tmap(&tmW, wg, C, H, rs::gemm_b_box_rows(bn, pair)));
   RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
   p.K = C;
   p.n_blocks = H / bn;
-  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.num_tiles = rs::gemm_num_tiles(M, p.n_blocks, pair);
   p.stats = reinterpret_cast<const float2*>(stats);
   p.colG = colg;
   p.colC = colc;
@@ -396,7 +400,7 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   p.err = st->err;
   p.timeout_ns = static_cast<unsigned long long>(timeout_us) * 1000ull;
   p.debug_skip_kb = skip_kblock;
-  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, st->num_sms, s));
+  RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, pair, st->num_sms, s));
   return RS_OK;
 }
 

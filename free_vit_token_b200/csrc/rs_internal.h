@@ -29,25 +29,42 @@ constexpr int kFc2PartialsPerTile = 2;
 // Launches `kern` on `stream`; with `pdl` the launch may begin while the
 // previous kernel in the stream is still running (every kernel of this library
 // waits for its predecessor with griddepcontrol.wait before touching memory).
+// With `cluster` > 1 the grid is cut into clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                          cudaStream_t stream, bool pdl, Args&&... args) {
+inline cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, bool pdl, int cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = pdl ? attr : nullptr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = n > 0 ? attr : nullptr;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool pdl, Args&&... args) {
+  return launch_cluster(kern, grid, block, smem, stream, pdl, 1, static_cast<Args&&>(args)...);
 }
 
 struct MlpParams {
   int M, N, K;                    // output rows, output columns, reduction length
-  int n_blocks, num_tiles;        // N / BN, ceil(M / 128) * n_blocks
+  int n_blocks, num_tiles;        // N / BN, gemm_num_tiles(M, n_blocks, pair)
   const __nv_bfloat16* ln_gamma;  // [K]   fc1 only
   const __nv_bfloat16* ln_beta;   // [K]   fc1 only
   const float2* stats;            // [M]   fc1 only: (mean, rstd) per row
@@ -64,7 +81,21 @@ struct MlpParams {
                                   // first tile (-1: off)
 };
 
-size_t mlp_smem_bytes(int bn, bool ln, int epi, int K);
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);
+
+// CTA pairs (tcgen05 cta_group::2, 256-row tiles with B split between the two
+// CTAs) for long reductions (K >= 1024: fc2, and fc1 at C >= 1024), where the
+// third less operand traffic per CTA pays; single CTAs (128-row tiles) for short
+// K, where the epilogue bounds the kernel and one tile per SM (148 units rather
+// than the resident pairs) splits the grid into fewer waves. Not for the
+// staged-LN kernel.
+inline bool gemm_pair(int M, int K, bool staged_ln) { return !staged_ln && M > 128 && K >= 1024; }
+inline int gemm_num_tiles(int M, int n_blocks, bool pair) {
+  const int tm = pair ? 256 : 128;
+  return ((M + tm - 1) / tm) * n_blocks;
+}
+// Rows of the B tile one CTA loads (its tensor map's box height).
+inline int gemm_b_box_rows(int bn, bool pair) { return pair ? bn / 2 : bn; }
 int fc1_block_n(int H);
 int fc2_block_n(int C);
 cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
@@ -77,17 +108,20 @@ cudaError_t launch_ln_prep(const void* x, int M, int C, float* stats, const void
                            const void* gamma, const void* beta, const void* b1, int H, void* Wg,
                            float* colG, float* colC, int num_sms, cudaStream_t stream,
                            bool pdl = false);
+// `pair`: CTA-pair kernel (p.num_tiles and tmW1's box from gemm_num_tiles and
+// gemm_b_box_rows with the same flag); not with staged_ln.
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s,
-                       bool pdl = false);
+                       const MlpParams& p, int bn, bool staged_ln, bool pair, int num_sms,
+                       cudaStream_t s, bool pdl = false);
 cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream);
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
-                       const MlpParams& p, int bn, int num_sms, cudaStream_t s, bool pdl = false);
+                       const MlpParams& p, int bn, bool pair, int num_sms, cudaStream_t s,
+                       bool pdl = false);
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
                           float* scores, int32_t* kept_idx, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
                           void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);
-// Selection then gather: one fused kernel for L <= 256, else the two kernels above.
+// Selection then gather in one kernel (B x S CTAs; every CTA of a sample selects).
 cudaError_t launch_select_gather(const float* partials, int num_partials, const void* y, int B,
                                  int L, int C, int keep_k, float* scores, int32_t* kept_idx,
                                  void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);

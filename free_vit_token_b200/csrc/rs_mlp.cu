@@ -42,7 +42,11 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr int kVecMaxBytes = 2 * 256 * 4;       // one tile's column vectors (fold: G and cb)
 
-__host__ __device__ constexpr int stage_bytes(int bn) { return kAStageBytes + bn * kBK * 2; }
+// One pipeline stage: the A tile (128 rows) and this CTA's rows of the B tile
+// (all BN, or BN / 2 when a CTA pair shares the tile).
+__host__ __device__ constexpr int stage_bytes(int bn, bool pair) {
+  return kAStageBytes + (pair ? bn / 2 : bn) * kBK * 2;
+}
 // Per-tile column vectors the epilogue reads: the folded-LN G and cb (fp32) or
 // the bias (bf16), for BN columns; double-buffered with the accumulator.
 __host__ __device__ constexpr int vec_bytes(int bn, int epi) {
@@ -57,10 +61,10 @@ __host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
   return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + kMaxEpiWarps * kEpiBoxBytes +
          2 * kVecMaxBytes;
 }
-__host__ __device__ constexpr int num_stages(int bn, bool ln, int epi) {
-  return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn) > 6
-             ? 6
-             : (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn);
+__host__ __device__ constexpr int num_stages(int bn, bool ln, int epi, bool pair) {
+  return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn, pair) > (pair ? 8 : 6)
+             ? (pair ? 8 : 6)
+             : (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn, pair);
 }
 // Epilogue warps EW: 8 (two per TMEM lane quadrant) or 16 (four). 16 pays off
 // only where the epilogue's arithmetic rivals a short main loop (fc1 with
@@ -69,8 +73,8 @@ __host__ __device__ constexpr int num_threads(bool ln, int ew) {
   return (kEpiWarp0 + ew + (ln ? kNumLnWarps : 0)) * 32;
 }
 
-size_t mlp_smem_bytes(int bn, bool ln, int epi, int K) {
-  return 1024 + static_cast<size_t>(num_stages(bn, ln, epi)) * stage_bytes(bn) +
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair) {
+  return 1024 + static_cast<size_t>(num_stages(bn, ln, epi, pair)) * stage_bytes(bn, pair) +
          kMaxEpiWarps * kEpiBoxBytes + 2 * vec_stride(bn, epi) + kCtrlBytes +
          (ln ? 4 * static_cast<size_t>(K) : 0);
 }
@@ -173,13 +177,18 @@ cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
-template <int BN, bool LN_A, int EPI, int EW>
+template <int BN, bool LN_A, int EPI, int EW, bool PAIR>
 __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     mlp_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const MlpParams p) {
-  constexpr int kBStageBytes = BN * kBK * 2;
-  constexpr int STAGES = num_stages(BN, LN_A, EPI);
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN);
+  static_assert(!(PAIR && LN_A), "the staged-LN kernel runs on single CTAs");
+  constexpr int kBRows = PAIR ? BN / 2 : BN;       // rows of the B tile this CTA loads
+  constexpr int kBStageBytes = kBRows * kBK * 2;
+  constexpr int STAGES = num_stages(BN, LN_A, EPI, PAIR);
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;      // output rows of one tile
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN);
+  // bytes that complete one stage's full barrier (the leader's, for a pair)
+  constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kAStageBytes + kBStageBytes);
   constexpr int kNumEpiWarps = EW;
   static_assert(EW == 8 || EW == 16, "epilogue warps");
   static_assert(!LN_A || EW == 8, "staged-LN kernel: 8 epilogue warps");
@@ -214,6 +223,14 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int KB = p.K / kBK;
+  // A CTA pair (a cluster of two) shares each tile: CTA `rank` holds A rows
+  // 128 * rank .. +127 of the 256-row tile and B rows BN/2 * rank .. +BN/2-1; the
+  // leader (rank 0) issues the MMAs, whose accumulator rows land in the TMEM of
+  // the CTA that holds them.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -223,7 +240,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kNumEpiWarps);
+      mbar_init(&tempty[a], PAIR ? 2 * kNumEpiWarps : kNumEpiWarps);
       mbar_init(&vfull[a], 1);
       mbar_init(&vempty[a], kNumEpiWarps);
     }
@@ -237,8 +254,13 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   // Nothing above touched global memory: let the next kernel launch, then wait
   // for the previous one to finish before reading anything it may have written.
@@ -253,7 +275,11 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
@@ -269,7 +295,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
       int vpend0 = -1, vpend1 = -1;
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) pend[s] = -1;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = unit0; tile < p.num_tiles; tile += units) {
         const int m_blk = tile / p.n_blocks, n_blk = tile % p.n_blocks;
         // this tile's column vectors, into the buffer of the accumulator it will use
         if (!wait_bounded(&vempty[vacc], vphase ^ 1u, wc)) break;
@@ -287,14 +313,25 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, wc)) { ok = false; break; }
           // test hook: leave one stage unfilled so the consumer's wait runs out
-          const bool skip = kb == p.debug_skip_kb && blockIdx.x == 0 && tile == blockIdx.x;
+          const bool skip = kb == p.debug_skip_kb && blockIdx.x == 0 && tile == unit0;
           if (!skip) {
-            mbar_arrive_expect_tx(&full[stage], stage_bytes(BN));
-            tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, m_blk * kBM);
-            tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, n_blk * BN);
+            if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
+            if constexpr (PAIR) {
+              // both CTAs' loads complete on the leader's full barrier
+              const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0u);
+              tma_load_2d_pair(sA + stage * kAStageBytes, &tmA, fb, kb * kBK,
+                               m_blk * kTileM + static_cast<int>(rank) * kBM);
+              tma_load_2d_pair(sB + stage * kBStageBytes, &tmB, fb, kb * kBK,
+                               n_blk * BN + static_cast<int>(rank) * kBRows);
+            } else {
+              tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, m_blk * kBM);
+              tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, n_blk * BN);
+            }
+            if (leader) {
 #pragma unroll
-            for (int s = 0; s < STAGES; ++s)
-              if (s == stage) pend[s] = static_cast<int>(phase);
+              for (int s = 0; s < STAGES; ++s)
+                if (s == stage) pend[s] = static_cast<int>(phase);
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -306,18 +343,27 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         if (pend[s] >= 0) wait_bounded(&full[s], static_cast<uint32_t>(pend[s]), wc, false);
       if (vpend0 >= 0) wait_bounded(&vfull[0], static_cast<uint32_t>(vpend0), wc, false);
       if (vpend1 >= 0) wait_bounded(&vfull[1], static_cast<uint32_t>(vpend1), wc, false);
+      if constexpr (PAIR) {
+        // The leader's releases of every stage (multicast commits into this CTA's
+        // empty barriers) have all arrived before the CTA may exit.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, wc)) break;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, wc)) break;
+      for (int tile = unit0; tile < p.num_tiles; tile += units) {
+        // a pair's tempty also counts the peer's epilogue warps (remote arrivals)
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, wc, true, PAIR)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         bool ok = true;
@@ -328,19 +374,32 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
           const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * kAStageBytes));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * kBStageBytes));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(d_tmem, ad + 2u * k, bd + 2u * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k) {
+            if constexpr (PAIR)
+              umma_bf16_pair(d_tmem, ad + 2u * k, bd + 2u * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, ad + 2u * k, bd + 2u * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
           issued = true;
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR)
+            umma_commit_pair_mc(&empty[stage], 0x3);  // both CTAs' producers
+          else
+            umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR)
+          umma_commit_pair_mc(&tfull[acc], 0x3);  // both CTAs' epilogues
+        else
+          umma_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       if (*abort_flag && issued) {
         // Drain: wait until every MMA issued so far has finished with TMEM and smem.
-        umma_commit(drain);
+        if constexpr (PAIR)
+          umma_commit_pair(drain);
+        else
+          umma_commit(drain);
         wait_bounded(drain, 0u, wc, false);
       }
     }
@@ -364,8 +423,9 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     const uint32_t box_u32 = smem_u32(box);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = unit0; tile < p.num_tiles; tile += units) {
       const int m_blk = tile / p.n_blocks, n_blk = tile % p.n_blocks;
+      const int row0 = m_blk * kTileM + static_cast<int>(rank) * kBM;  // this CTA's first row
       int ok = 1;
       if (lane == 0)
         ok = (wait_bounded(&vfull[acc], acc_phase, wc) && wait_bounded(&tfull[acc], acc_phase, wc))
@@ -376,8 +436,9 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
       mbar_try_wait(&vfull[acc], acc_phase);  // completed: acquire for every lane
       mbar_try_wait(&tfull[acc], acc_phase);
       tc_fence_after_sync();
-      const int row = m_blk * kBM + q * 32 + lane;
+      const int row = row0 + q * 32 + lane;
       const bool row_ok = row < p.M;
+      const bool box_live = row0 + q * 32 < p.M;  // the warp's box holds rows of the output
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + grp * kCols);
       const int col0 = n_blk * BN + grp * kCols;
@@ -420,7 +481,12 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         } else {
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) {
+            if (PAIR && !leader)
+              mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0u));
+            else
+              mbar_arrive(&tempty[acc]);
+          }
         }
         const int c = n * 16;
         const uint32_t cvec = grp * kCols + c;  // column of this chunk within the tile
@@ -500,8 +566,8 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
                make_uint4(outw[4], outw[5], outw[6], outw[7]));
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmOut, box, col0 + c, m_blk * kBM + q * 32);
+        if (lane == 0 && box_live) {
+          tma_store_2d(&tmOut, box, col0 + c, row0 + q * 32);
           bulk_commit_group();
         }
       }
@@ -529,7 +595,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+    for (int tile = unit0; tile < p.num_tiles && ok; tile += units) {
       const int m_blk = tile / p.n_blocks;
       uint64_t rs2[8], nm2[8];  // (rstd, rstd) and (-mean*rstd, -mean*rstd) per row
 #pragma unroll
@@ -586,24 +652,62 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
   }
 
   __syncthreads();
+  if constexpr (PAIR) {
+    // After an abort a CTA may still have loads in flight that complete on the
+    // other CTA's barriers and that neither CTA can wait for: give them time to
+    // land. Then neither CTA leaves (or frees TMEM) before the other is done.
+    if (threadIdx.x == 0 && (*abort_flag || *reinterpret_cast<volatile int*>(p.err) != 0))
+      spin_ns(1000000);
+    cluster_sync();
+  }
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int BN, bool LN_A, int EPI, int EW = 8>
+template <int BN, bool LN_A, int EPI, int EW = 8, bool PAIR = false>
 static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                const CUtensorMap& tmOut, const MlpParams& p, int num_sms,
                                cudaStream_t stream, bool pdl) {
-  auto kern = mlp_gemm_kernel<BN, LN_A, EPI, EW>;
-  const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K);
+  auto kern = mlp_gemm_kernel<BN, LN_A, EPI, EW, PAIR>;
+  const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K, PAIR);
+  const int threads = num_threads(LN_A, EW);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  return launch(kern, grid, num_threads(LN_A, EW), smem, stream, pdl, tmA, tmB, tmOut, p);
+  if constexpr (PAIR) {
+    // One CTA pair per two SMs, as many pairs as can be resident at once (an SM
+    // whose partner in its GPC is missing stays idle).
+    static const int max_pairs = [&]() {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (num_sms / 2));
+      cfg.blockDim = dim3(threads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms / 2;
+      }
+      return n < num_sms / 2 ? n : num_sms / 2;
+    }();
+    const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
+    return launch_cluster(kern, 2 * pairs, threads, smem, stream, pdl, 2, tmA, tmB, tmOut, p);
+  } else {
+    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    return launch(kern, grid, threads, smem, stream, pdl, tmA, tmB, tmOut, p);
+  }
 }
 
 int fc1_block_n(int H) { return H % 256 == 0 ? 256 : (H % 128 == 0 ? 128 : 64); }
@@ -611,10 +715,20 @@ int fc2_block_n(int C) {
   return C % 256 == 0 ? 256 : (C % 192 == 0 ? 192 : (C % 128 == 0 ? 128 : 64));
 }
 
+template <int BN, int EW>
+static cudaError_t launch_fold(const CUtensorMap& tmX, const CUtensorMap& tmW1,
+                               const CUtensorMap& tmHid, const MlpParams& p, bool pair,
+                               int num_sms, cudaStream_t s, bool pdl) {
+  return pair ? launch_gemm<BN, false, kEpiGeluFold, EW, true>(tmX, tmW1, tmHid, p, num_sms, s, pdl)
+              : launch_gemm<BN, false, kEpiGeluFold, EW, false>(tmX, tmW1, tmHid, p, num_sms, s,
+                                                                  pdl);
+}
+
 cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CUtensorMap& tmHid,
-                       const MlpParams& p, int bn, bool staged_ln, int num_sms, cudaStream_t s,
-                       bool pdl) {
+                       const MlpParams& p, int bn, bool staged_ln, bool pair, int num_sms,
+                       cudaStream_t s, bool pdl) {
   if (staged_ln) {
+    if (pair) return cudaErrorInvalidValue;
     switch (bn) {
       case 256: return launch_gemm<256, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
       case 128: return launch_gemm<128, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
@@ -623,25 +737,35 @@ cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CU
   }
   if (p.K <= 512) {
     switch (bn) {
-      case 256: return launch_gemm<256, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
-      case 128: return launch_gemm<128, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
-      default: return launch_gemm<64, false, kEpiGeluFold, 16>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+      case 256: return launch_fold<256, 16>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
+      case 128: return launch_fold<128, 16>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
+      default: return launch_fold<64, 16>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
     }
   }
   switch (bn) {
-    case 256: return launch_gemm<256, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
-    case 128: return launch_gemm<128, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
-    default: return launch_gemm<64, false, kEpiGeluFold>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
+    case 256: return launch_fold<256, 8>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
+    case 128: return launch_fold<128, 8>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
+    default: return launch_fold<64, 8>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
   }
 }
 
+template <int BN>
+static cudaError_t launch_resid(const CUtensorMap& tmHid, const CUtensorMap& tmW2,
+                                const CUtensorMap& tmY, const MlpParams& p, bool pair, int num_sms,
+                                cudaStream_t s, bool pdl) {
+  return pair ? launch_gemm<BN, false, kEpiResidShift, 8, true>(tmHid, tmW2, tmY, p, num_sms, s, pdl)
+              : launch_gemm<BN, false, kEpiResidShift, 8, false>(tmHid, tmW2, tmY, p, num_sms, s,
+                                                                   pdl);
+}
+
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
-                       const MlpParams& p, int bn, int num_sms, cudaStream_t s, bool pdl) {
+                       const MlpParams& p, int bn, bool pair, int num_sms, cudaStream_t s,
+                       bool pdl) {
   switch (bn) {
-    case 256: return launch_gemm<256, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
-    case 192: return launch_gemm<192, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
-    case 128: return launch_gemm<128, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
-    default: return launch_gemm<64, false, kEpiResidShift>(tmHid, tmW2, tmY, p, num_sms, s, pdl);
+    case 256: return launch_resid<256>(tmHid, tmW2, tmY, p, pair, num_sms, s, pdl);
+    case 192: return launch_resid<192>(tmHid, tmW2, tmY, p, pair, num_sms, s, pdl);
+    case 128: return launch_resid<128>(tmHid, tmW2, tmY, p, pair, num_sms, s, pdl);
+    default: return launch_resid<64>(tmHid, tmW2, tmY, p, pair, num_sms, s, pdl);
   }
 }
 

@@ -135,7 +135,8 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
   p.err = err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
-  if (rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, num_sms, st) != cudaSuccess) {
+  // single-CTA tiles: p.num_tiles and tmW's box above are the 128-row forms
+  if (rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, /*pair=*/false, num_sms, st) != cudaSuccess) {
     cudaGetLastError();
     return RS_ERR_CUDA;
   }

@@ -53,6 +53,37 @@ __device__ __forceinline__ uint32_t block_exclusive_count(bool flag, uint32_t* s
   return res;
 }
 
+// Exclusive prefix sum of `v` over the block in thread order; `total` receives
+// the block-wide sum. Every thread of the block must call it.
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t* s_warp,
+                                                        uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = lane < nw ? s_warp[lane] : 0u;
+    uint32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    s_warp[lane] = wi - w;
+    if (lane == 31) s_warp[32] = wi;
+  }
+  __syncthreads();
+  const uint32_t res = s_warp[warp] + incl - v;
+  total = s_warp[32];
+  __syncthreads();
+  return res;
+}
+
 // Number of patch tokens u in 1..L-1 that beat key `key` of token t (t >= 1):
 // key_u >= key for u < t, key_u > key for u > t (u = t never counts). The sweep
 // is split at t so every key costs one compare. s_key holds L keys padded with
@@ -110,12 +141,24 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
                                           float* __restrict__ scores, const SelSmem& s) {
   const int Lpad = (L + 3) & ~3;
   const float* P = partials + static_cast<size_t>(b) * L * NP;
+  // An even NP (what fc2 writes) keeps every row 8-byte aligned: pairs of loads.
+  const bool pairs = (NP & 1) == 0;
   for (int t = threadIdx.x; t < Lpad; t += blockDim.x) {
     uint32_t key = 0;
     if (t < L) {
       const float* pr = P + static_cast<size_t>(t) * NP;
-      float acc = 0.f;
-      for (int j = 0; j < NP; ++j) acc += pr[j];
+      float acc = 0.f;  // left to right
+      if (pairs) {
+        const float2* pr2 = reinterpret_cast<const float2*>(pr);
+#pragma unroll 4
+        for (int j = 0; j < (NP >> 1); ++j) {
+          const float2 v2 = __ldg(pr2 + j);
+          acc += v2.x;
+          acc += v2.y;
+        }
+      } else {
+        for (int j = 0; j < NP; ++j) acc += __ldg(pr + j);
+      }
       const float v = sqrtf(acc);
       if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
       key = __float_as_uint(v);
@@ -146,18 +189,26 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
     __syncthreads();
     return;
   }
-  // Radix select of the k-th largest key among t = 1..L-1.
+  // Radix select of the k-th largest key among t = 1..L-1. Each round of a pass
+  // gives thread tid the four keys t = base + 4 tid .. +3 (one 16-byte load).
+  const int Lpad = (L + 3) & ~3;
+  const uint4* key4 = reinterpret_cast<const uint4*>(s.key);
   uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += nt) s.hist[i] = 0;
     __syncthreads();
-    for (int base = 1; base < L; base += nt) {
-      const int t = base + tid;
-      const uint32_t u = t < L ? s.key[t] : 0u;
-      const bool cand = t < L && (u & mask) == prefix;
-      const uint32_t digit = cand ? ((u >> shift) & 0xFFu) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
+    for (int base = 0; base < L; base += 4 * nt) {
+      const int t0 = base + 4 * tid;
+      const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
+      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        const bool cand = t >= 1 && t < L && (u[i] & mask) == prefix;
+        const uint32_t digit = cand ? ((u[i] >> shift) & 0xFFu) : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+        if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
+      }
     }
     __syncthreads();
     if (warp == 0) {
@@ -188,26 +239,44 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
       }
     }
     __syncthreads();
+    // s.sel is rewritten only after the next pass's first barrier: no barrier here
     prefix |= s.sel[0] << shift;
     mask |= 0xFFu << shift;
     need -= s.sel[1];
-    __syncthreads();
   }
-  const uint32_t T = prefix;  // k-th largest key; `need` keys equal to T are kept
-  uint32_t eq_base = 0, out_base = 0;
-  for (int base = 1; base < L; base += nt) {
-    const int t = base + tid;
-    const bool valid = t < L;
-    const uint32_t u = valid ? s.key[t] : 0u;
-    const bool gt = valid && u > T;
-    const bool eq = valid && u == T;
-    uint32_t eq_tot, keep_tot;
-    const uint32_t eq_rank = eq_base + block_exclusive_count(eq, s.warp, eq_tot);
-    const bool keep = gt || (eq && eq_rank < need);
-    const uint32_t pos = out_base + block_exclusive_count(keep, s.warp, keep_tot);
-    if (keep) s.kept[1 + pos] = t;
-    eq_base += eq_tot;
-    out_base += keep_tot;
+  // Ordered compaction: token t (1 <= t < L) is kept when key_t > T, or key_t == T
+  // and fewer than `need` equal keys precede it; its place among the kept tokens
+  // is (#keys > T before t) + min(#keys == T before t, need). One packed scan per
+  // round counts both (> T in the low half, == T in the high half).
+  const uint32_t T = prefix;  // the k-th largest key
+  uint32_t gt_base = 0, eq_base = 0;
+  for (int base = 0; base < L; base += 4 * nt) {
+    const int t0 = base + 4 * tid;
+    const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
+    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+    uint32_t gt_m = 0, eq_m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + i;
+      if (t >= 1 && t < L) {
+        gt_m |= static_cast<uint32_t>(u[i] > T) << i;
+        eq_m |= static_cast<uint32_t>(u[i] == T) << i;
+      }
+    }
+    uint32_t tot;
+    const uint32_t pre =
+        block_exclusive_sum(static_cast<uint32_t>(__popc(gt_m)) | (static_cast<uint32_t>(__popc(eq_m)) << 16),
+                            s.warp, tot);
+    uint32_t gtb = gt_base + (pre & 0xFFFFu), eqb = eq_base + (pre >> 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t gt = (gt_m >> i) & 1u, eq = (eq_m >> i) & 1u;
+      if (gt || (eq && eqb < need)) s.kept[1 + gtb + (eqb < need ? eqb : need)] = t0 + i;
+      gtb += gt;
+      eqb += eq;
+    }
+    gt_base += tot & 0xFFFFu;
+    eq_base += tot >> 16;
   }
   __syncthreads();
 }
@@ -272,8 +341,10 @@ __device__ __forceinline__ void copy_rows(const uint4* __restrict__ y, int L, in
 // j0, j0 + S, ... of them; CTA (b, 0) also writes scores and kept_idx.
 constexpr int kSelGatherThreads = 512;
 
+// Two CTAs per SM, except for the widest rows (C > 1024), whose 32 registers of
+// row data per lane need more than half of an SM's register file.
 template <int VPL>
-__global__ void __launch_bounds__(kSelGatherThreads, 2) select_gather_kernel(
+__global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_gather_kernel(
     const float* __restrict__ partials, int NP, int L, int k, const uint4* __restrict__ y, int Cv,
     int S, float* __restrict__ scores, int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];

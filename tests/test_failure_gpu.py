@@ -12,12 +12,13 @@ from workloads import random_block
 pytestmark = pytest.mark.gpu
 
 
-def test_withheld_load_times_out_and_context_survives():
+@pytest.mark.parametrize("M,C,H", [(300, 384, 1536),    # single-CTA tiles
+                                   (300, 1024, 4096)])  # CTA-pair tiles (K >= 1024)
+def test_withheld_load_times_out_and_context_survives(M, C, H):
     import free_vit_token_b200 as rs
     import free_vit_token_b200.rs as rsmod
 
     dev = torch.device("cuda:0")
-    M, C, H = 300, 384, 1536
     inp = random_block(1, M, C, H, seed=31, fg_rows=20)
     x = inp.x.reshape(M, C).to(dev)
     w = inp.weights[0]
