@@ -38,6 +38,9 @@ from workloads import WORKLOADS, make_inputs  # noqa: E402
 METRIC = "pruned-MLP-block tokens/sec at 1 B200; % of bf16 tensor peak; select+gather GB/s"
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
+SG_REPS = 20  # select+gather launches per timing graph
+
+
 def kernels_per_step(wl) -> int:
     """Kernels rs_block_forward launches per stage: LN prep (statistics + weight
     fold), fc1, fc2, then one fused select+gather kernel (L <= 256) or select and
@@ -336,7 +339,35 @@ def main():
     dominant = max(fc_ms, key=fc_ms.get)
     flops = sum(gemm_flops.values())
     achieved_tf = flops / (fc_ms[dominant] / 1e3) / 1e12
-    sel_ms = sum(statistics.mean(per_stage[s]["select_gather"]) for s in per_stage)
+    sel_ms_event = sum(statistics.mean(per_stage[s]["select_gather"]) for s in per_stage)
+    # Device time of one select+gather launch: SG_REPS launches captured in a CUDA
+    # graph and replayed (launch overhead amortised). y and the partials are the
+    # ones fc2 just wrote in the breakdown above, L2-resident as in the block.
+    sel_ms = 0.0
+    cap_stream = torch.cuda.Stream(dev)
+    for s, k in enumerate(wl.keep_k):
+        L_s = wl.stage_L(s)
+        M = wl.B * L_s
+        y2 = ybuf[: M * wl.C].view(wl.B, L_s, wl.C)
+        p2 = pbuf[: M * np_].view(M, np_)
+        cap_stream.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            for _ in range(SG_REPS):
+                rs.rs_select_gather(p2, y2, k, scores=outs[s][2], kept_idx=outs[s][1],
+                                    y_kept=outs[s][0], stream=cap_stream)
+        g.replay()  # replays run on the current stream (`stream`)
+        torch.cuda.synchronize()
+        reps = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            reps.append(a.elapsed_time(b) / SG_REPS)
+        sel_ms += statistics.median(reps)
+        del g
     sg_bytes = 0
     for s, k in enumerate(wl.keep_k):
         M = wl.tokens(s)
@@ -394,7 +425,10 @@ def main():
         "kernel_ms": {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage)
                       for n in names},
         "select_gather": {"GBps": sg_gbs, "frac_hbm": sg_gbs / peaks["hbm"],
-                          "bytes": sg_bytes, "ms": sel_ms},
+                          "bytes": sg_bytes, "ms": sel_ms,
+                          "timing": f"device time per launch, {SG_REPS} launches replayed from a "
+                                    "CUDA graph, inputs as fc2 left them (L2-resident)",
+                          "ms_single_launch_events": sel_ms_event},
         "images_per_s": world * wl.B / (ms_per_step / 1e3),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

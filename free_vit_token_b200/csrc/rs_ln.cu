@@ -2,8 +2,8 @@
 // "Representation Shift: Unifying Token Compression with FlashAttention"):
 //
 //   ln_stats:  per row r of x', mean_r and rstd_r = 1/sqrt(var_r + eps) (biased
-//              variance), one warp per row, two passes over the row held in
-//              registers, reductions by warp shuffles.
+//              variance), 8, 16 or 32 lanes per row by width, two passes over
+//              the row held in registers, reductions by shuffles.
 //   ln_fold:   the LayerNorm's affine part folded into fc1's weights. With
 //              u = (x' - mean) * rstd * gamma + beta,
 //                W1 u + b1 = rstd * (Wg x' - mean * G) + cb,
@@ -25,69 +25,77 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int VPL>
-__device__ __forceinline__ void load_row(const uint4* __restrict__ xr, int lane, int nvec,
-                                         uint4 (&v)[VPL]) {
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int idx = lane + 32 * i;
-    v[i] = idx < nvec ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
-  }
-}
-
-// Persistent: each warp walks rows with a grid-wide stride and keeps the next
-// row's loads in flight while it reduces the current one. `gw0`/`nw` are this
-// warp's index and the warp count of the part of the grid doing this work.
-template <int VPL>
+// Persistent: each warp takes 32 / LPR rows per step (LPR lanes per row, VPL
+// 16-byte vectors per lane at most), walks the rows with a grid-wide stride and
+// keeps the next step's loads in flight while it reduces the current rows. Sums
+// run on pairs of fp32 lanes. `gw0`/`nw` are this warp's index and the warp
+// count of the part of the grid doing this work.
+template <int LPR, int VPL>
 __device__ __forceinline__ void ln_stats_body(const __nv_bfloat16* __restrict__ x, int M, int C,
                                               float2* __restrict__ stats, int gw0, int nw) {
+  constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
-  int row = gw0;
+  const int sub = lane / LPR, l = lane % LPR;
   const int nvec = C >> 3;
   const float inv_c = 1.0f / static_cast<float>(C);
+  auto load = [&](int r, uint4(&v)[VPL]) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * C);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int idx = l + LPR * i;
+      v[i] = (r < M && idx < nvec) ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
+    }
+  };
   uint4 cur[VPL], nxt[VPL];
-  if (row < M) load_row<VPL>(reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * C), lane,
-                             nvec, cur);
-  for (; row < M; row += nw) {
-    const int nrow = row + nw;
-    if (nrow < M)
-      load_row<VPL>(reinterpret_cast<const uint4*>(x + static_cast<size_t>(nrow) * C), lane, nvec,
-                    nxt);
-    float sum = 0.f;
+  const int step = nw * RPW;
+  int base = gw0 * RPW;
+  if (base < M) load(base + sub, cur);
+  for (; base < M; base += step) {
+    const int row = base + sub;
+    if (base + step < M) load(base + step + sub, nxt);
+    uint64_t s2 = 0;  // padding vectors are zero: they add nothing
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const uint32_t* w = reinterpret_cast<const uint32_t*>(&cur[i]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sum += bf16lo(w[e]) + bf16hi(w[e]);
+      for (int e = 0; e < 4; ++e) s2 = fadd2(s2, bf16x2_to_f2(w[e]));
     }
-    const float mean = warp_sum(sum) * inv_c;
-    float sq = 0.f;
+    float2 sf = f2unpack(s2);
+    float sum = sf.x + sf.y;
+#pragma unroll
+    for (int o = LPR / 2; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mean = sum * inv_c;
+    const uint64_t nm2 = f2pack(-mean, -mean);
+    uint64_t q2 = 0;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      if (lane + 32 * i < nvec) {
+      if (l + LPR * i < nvec) {
         const uint32_t* w = reinterpret_cast<const uint32_t*>(&cur[i]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float d0 = bf16lo(w[e]) - mean, d1 = bf16hi(w[e]) - mean;
-          sq = fmaf(d0, d0, sq);
-          sq = fmaf(d1, d1, sq);
+          const uint64_t d2 = fadd2(bf16x2_to_f2(w[e]), nm2);
+          q2 = ffma2(d2, d2, q2);
         }
       }
     }
-    sq = warp_sum(sq);
-    if (lane == 0) stats[row] = make_float2(mean, rsqrtf(sq * inv_c + kLnEps));
+    const float2 qf = f2unpack(q2);
+    float sq = qf.x + qf.y;
+#pragma unroll
+    for (int o = LPR / 2; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (l == 0 && row < M) stats[row] = make_float2(mean, rsqrtf(sq * inv_c + kLnEps));
 #pragma unroll
     for (int i = 0; i < VPL; ++i) cur[i] = nxt[i];
   }
 }
 
-template <int VPL>
+template <int LPR, int VPL>
 __global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int M,
                                                        int C, float2* __restrict__ stats) {
   pdl_trigger();
   pdl_wait();
-  ln_stats_body<VPL>(x, M, C, stats, static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5),
-                     static_cast<int>((gridDim.x * blockDim.x) >> 5));
+  ln_stats_body<LPR, VPL>(x, M, C, stats,
+                          static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5),
+                          static_cast<int>((gridDim.x * blockDim.x) >> 5));
 }
 
 template <int VPL>
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // Both in one grid: the first `stats_blocks` blocks compute statistics, the rest fold.
-template <int VPL>
+template <int VPL, int LPR, int SVPL>
 __global__ void __launch_bounds__(256)
     ln_prep_kernel(const __nv_bfloat16* __restrict__ x, int M, float2* __restrict__ stats,
                    int stats_blocks, const __nv_bfloat16* __restrict__ W1,
@@ -168,7 +176,7 @@ __global__ void __launch_bounds__(256)
   const int wpb = blockDim.x >> 5;
   const int w = threadIdx.x >> 5;
   if (static_cast<int>(blockIdx.x) < stats_blocks) {
-    ln_stats_body<VPL>(x, M, C, stats, blockIdx.x * wpb + w, stats_blocks * wpb);
+    ln_stats_body<LPR, SVPL>(x, M, C, stats, blockIdx.x * wpb + w, stats_blocks * wpb);
   } else {
     const int fb = blockIdx.x - stats_blocks;
     ln_fold_body<VPL>(W1, gamma, beta, b1, H, C, Wg, colG, colC, fb * wpb + w,
@@ -176,8 +184,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-static int stats_blocks_for(int M, int num_sms) {
-  const int warps = (M + 1) / 2;  // two rows per warp on average keeps loads in flight
+static int stats_blocks_for(int M, int C, int num_sms) {
+  const int rpw = C <= 256 ? 4 : (C <= 512 ? 2 : 1);  // rows per warp step
+  const int warps = (M + 2 * rpw - 1) / (2 * rpw);    // about two steps per warp
   int blocks = (warps + 7) / 8;
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   return blocks < 1 ? 1 : blocks;
@@ -190,13 +199,13 @@ static int fold_blocks_for(int H, int num_sms) {
 
 cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
                             cudaStream_t stream, bool pdl) {
-  const int blocks = stats_blocks_for(M, num_sms);
+  const int blocks = stats_blocks_for(M, C, num_sms);
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* sp = reinterpret_cast<float2*>(stats);
-  if (C <= 256) return launch(ln_stats_kernel<1>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
-  if (C <= 512) return launch(ln_stats_kernel<2>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
-  if (C <= 1024) return launch(ln_stats_kernel<4>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
-  return launch(ln_stats_kernel<8>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  if (C <= 256) return launch(ln_stats_kernel<8, 4>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  if (C <= 512) return launch(ln_stats_kernel<16, 4>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  if (C <= 1024) return launch(ln_stats_kernel<32, 4>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
+  return launch(ln_stats_kernel<32, 8>, blocks, 256, 0, stream, pdl, xp, M, C, sp);
 }
 
 cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,
@@ -220,7 +229,7 @@ cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, 
 cudaError_t launch_ln_prep(const void* x, int M, int C, float* stats, const void* W1,
                            const void* gamma, const void* beta, const void* b1, int H, void* Wg,
                            float* colG, float* colC, int num_sms, cudaStream_t stream, bool pdl) {
-  const int sb = stats_blocks_for(M, num_sms);
+  const int sb = stats_blocks_for(M, C, num_sms);
   const int fb = fold_blocks_for(H, num_sms);
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* sp = reinterpret_cast<float2*>(stats);
@@ -231,15 +240,15 @@ cudaError_t launch_ln_prep(const void* x, int M, int C, float* stats, const void
   auto* o = static_cast<__nv_bfloat16*>(Wg);
   const dim3 grid(sb + fb);
   if (C <= 256)
-    return launch(ln_prep_kernel<1>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+    return launch(ln_prep_kernel<1, 8, 4>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
                   colG, colC);
   if (C <= 512)
-    return launch(ln_prep_kernel<2>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+    return launch(ln_prep_kernel<2, 16, 4>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
                   colG, colC);
   if (C <= 1024)
-    return launch(ln_prep_kernel<4>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+    return launch(ln_prep_kernel<4, 32, 4>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
                   colG, colC);
-  return launch(ln_prep_kernel<8>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
+  return launch(ln_prep_kernel<8, 32, 8>, grid, 256, 0, stream, pdl, xp, M, sp, sb, w, g, b, bb, H, C, o,
                 colG, colC);
 }
 

@@ -137,33 +137,61 @@ __device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, 
 }
 
 // Scores of sample b from its partials into s.key (and to `scores` when given).
+// Each thread takes rows t = base + tid + i * nt (i < 4) per round and issues all
+// of their loads before adding; the fp32 additions of a row run left to right.
 __device__ __forceinline__ void load_keys(const float* __restrict__ partials, int NP, int L, int b,
                                           float* __restrict__ scores, const SelSmem& s) {
   const int Lpad = (L + 3) & ~3;
+  const int tid = threadIdx.x, nt = blockDim.x;
   const float* P = partials + static_cast<size_t>(b) * L * NP;
-  // An even NP (what fc2 writes) keeps every row 8-byte aligned: pairs of loads.
-  const bool pairs = (NP & 1) == 0;
-  for (int t = threadIdx.x; t < Lpad; t += blockDim.x) {
-    uint32_t key = 0;
-    if (t < L) {
-      const float* pr = P + static_cast<size_t>(t) * NP;
-      float acc = 0.f;  // left to right
-      if (pairs) {
-        const float2* pr2 = reinterpret_cast<const float2*>(pr);
-#pragma unroll 4
-        for (int j = 0; j < (NP >> 1); ++j) {
-          const float2 v2 = __ldg(pr2 + j);
-          acc += v2.x;
-          acc += v2.y;
-        }
-      } else {
-        for (int j = 0; j < NP; ++j) acc += __ldg(pr + j);
+  auto finish = [&](int t, float acc) {
+    const float v = sqrtf(acc);
+    if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
+    s.key[t] = __float_as_uint(v);
+  };
+  if ((NP & 1) == 0 && NP <= 8) {
+    // an even NP keeps every row 8-byte aligned: up to four pairs per row
+    const int np2 = NP >> 1;
+    const float2* P2 = reinterpret_cast<const float2*>(P);
+    for (int base = 0; base < Lpad; base += 4 * nt) {
+      float2 v[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = base + tid + i * nt;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          v[i][j] = (t < L && j < np2) ? __ldg(P2 + static_cast<size_t>(t) * np2 + j)
+                                       : make_float2(0.f, 0.f);
       }
-      const float v = sqrtf(acc);
-      if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
-      key = __float_as_uint(v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = base + tid + i * nt;
+        if (t < L) {
+          float acc = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < np2) {
+              acc += v[i][j].x;
+              acc += v[i][j].y;
+            }
+          }
+          finish(t, acc);
+        } else if (t < Lpad) {
+          s.key[t] = 0u;
+        }
+      }
     }
-    s.key[t] = key;
+  } else {
+    for (int t = tid; t < Lpad; t += nt) {
+      if (t < L) {
+        const float* pr = P + static_cast<size_t>(t) * NP;
+        float acc = 0.f;
+        for (int j = 0; j < NP; ++j) acc += __ldg(pr + j);
+        finish(t, acc);
+      } else {
+        s.key[t] = 0u;
+      }
+    }
   }
   __syncthreads();
 }
