@@ -41,11 +41,11 @@ FLUSH_BYTES = 256 << 20
 SG_REPS = 20  # select+gather launches per timing graph
 
 
-def kernels_per_step(wl, fused: bool) -> int:
+def kernels_per_step(wl) -> int:
     """Kernels rs_block_forward launches per stage: LN prep (statistics + weight
-    fold), the fused MLP kernel (narrow blocks) or fc1 and fc2, then one
-    select+gather kernel."""
-    return wl.stages * (3 if fused else 4)
+    fold), fc1, fc2, then one fused select+gather kernel (L <= 256) or select and
+    gather (longer L)."""
+    return sum(4 if wl.stage_L(s) <= 256 else 5 for s in range(wl.stages))
 
 
 def load_peaks():
@@ -61,7 +61,6 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- ncu traffic
 GEMM_SOURCES = ["free_vit_token_b200/csrc/rs_mlp.cu", "free_vit_token_b200/csrc/rs_ptx.cuh",
-                "free_vit_token_b200/csrc/rs_gelu.cuh", "free_vit_token_b200/csrc/rs_fused.cu",
                 "free_vit_token_b200/csrc/rs_gelu_poly.h", "free_vit_token_b200/csrc/rs_internal.h"]
 
 
@@ -291,11 +290,9 @@ def main():
     value = job_throughput(tokens_per_step, args.steps, total_ms, world)
 
     # ---- per-kernel breakdown (the same kernels, one step-level entry point each)
-    fused = rs.rs_mlp_fused_supported(wl.C, wl.H)
-    mlp_names = ("mlp_fused",) if fused else ("fc1", "fc2")
-    names = ("stats", "fold") + mlp_names + ("select_gather",)
+    names = ("stats", "fold", "fc1", "fc2", "select_gather")
     M0 = wl.tokens(0)
-    np_ = rs.RS_FUSED_PARTIALS if fused else rs.rs_num_partials(wl.C)  # partials per row
+    np_ = rs.rs_num_partials(wl.C)
     stats = torch.empty(M0, 2, dtype=torch.float32, device=dev)
     Wg = torch.empty(wl.H, wl.C, dtype=torch.bfloat16, device=dev)
     colG = torch.empty(wl.H, dtype=torch.float32, device=dev)
@@ -311,7 +308,7 @@ def main():
         for s, k in enumerate(wl.keep_k):
             L_s = wl.stage_L(s)
             M = wl.B * L_s
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
             x2 = xs.reshape(M, wl.C)
             st2 = stats[:M]
             h2 = hid[: M * wl.H].view(M, wl.H)
@@ -322,17 +319,13 @@ def main():
             e[1].record(stream)
             rs.rs_ln_fold(W[s][0], W[s][1], W[s][4], W[s][5], Wg, colG, colC, stream=stream)
             e[2].record(stream)
-            if fused:
-                rs.rs_mlp_fused(x2, st2, Wg, colG, colC, W[s][2], W[s][3], y=y2, partials=p2,
-                                stream=stream)
-            else:
-                rs.rs_fc1_gelu_folded(x2, st2, Wg, colG, colC, hidden=h2, stream=stream)
-                e[3].record(stream)
-                rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
-            e[len(names) - 1].record(stream)  # e[i] .. e[i + 1] brackets kernel names[i]
+            rs.rs_fc1_gelu_folded(x2, st2, Wg, colG, colC, hidden=h2, stream=stream)
+            e[3].record(stream)
+            rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
+            e[4].record(stream)
             rs.rs_select_gather(p2, y2.view(wl.B, L_s, wl.C), k, scores=outs[s][2],
                                 kept_idx=outs[s][1], y_kept=outs[s][0], stream=stream)
-            e[len(names)].record(stream)
+            e[5].record(stream)
             recs.append((s, e))
             xs = outs[s][0]
     torch.cuda.synchronize()
@@ -341,10 +334,8 @@ def main():
         d = per_stage.setdefault(s, {n: [] for n in names})
         for j, n in enumerate(names):
             d[n].append(e[j].elapsed_time(e[j + 1]))
-    # flops per launch: 2 M C H per GEMM; the fused kernel does both
-    gemm_flops = {s: 2.0 * wl.tokens(s) * wl.C * wl.H * (2 if fused else 1)
-                  for s in range(wl.stages)}
-    fc_ms = {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage) for n in mlp_names}
+    gemm_flops = {s: 2.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages)}
+    fc_ms = {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage) for n in ("fc1", "fc2")}
     dominant = max(fc_ms, key=fc_ms.get)
     flops = sum(gemm_flops.values())
     achieved_tf = flops / (fc_ms[dominant] / 1e3) / 1e12
@@ -423,9 +414,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config,
-        "roofline": {"bound": "tensor",
-                     "kernel": ("mlp_fused (tcgen05: fc1 + GELU + fc2 in one kernel)" if fused
-                                else f"{dominant} (tcgen05 GEMM)"),
+        "roofline": {"bound": "tensor", "kernel": f"{dominant} (tcgen05 GEMM)",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf,
                      "traffic": ncu_traffic(dominant, wl.name) if wl.stages == 1 else None,
@@ -443,7 +432,7 @@ def main():
         "images_per_s": world * wl.B / (ms_per_step / 1e3),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": kernels_per_step(wl, fused) * args.steps,
+        "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
     }

@@ -4,7 +4,6 @@ The compute lives in ``librs.so`` (CUDA kernels behind a C ABI, include/rs.h);
 ``free_vit_token_b200.rs`` is its ctypes binding.
 """
 from .rs import (  # noqa: F401
-    RS_FUSED_PARTIALS,
     RsError,
     lib,
     rs_block_forward,
@@ -19,8 +18,6 @@ from .rs import (  # noqa: F401
     rs_ln_fc1_gelu_noalloc,
     rs_ln_fc1_gelu_staged,
     rs_ln_stats,
-    rs_mlp_fused,
-    rs_mlp_fused_supported,
     rs_num_partials,
     rs_release_workspace,
     rs_select_gather,

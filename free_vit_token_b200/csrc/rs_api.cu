@@ -52,11 +52,8 @@ WsLayout ws_layout(int64_t M, int C, int H) {
   w.y = off;
   off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
   w.partials = off;
-  {
-    const int np_gemm = rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
-    const int np = np_gemm > rs::kFusedPartials ? np_gemm : rs::kFusedPartials;
-    off = align_up(off + static_cast<size_t>(M) * np * 4, 1024);
-  }
+  off = align_up(off + static_cast<size_t>(M) * (rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C)) * 4,
+                 1024);
   w.total = off;
   return w;
 }
@@ -228,32 +225,6 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
   RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, pair, st.num_sms, s, pdl));
-  return RS_OK;
-}
-
-// The fused MLP (rs_fused.cu) on LN statistics and folded weights already in place.
-int run_fused_step(DevState& st, const void* x, const float* stats, const void* wg,
-                   const float* colg, const float* colc, int M, int C, int H, const void* W2,
-                   const void* b2, void* y, float* partials, cudaStream_t s, bool pdl) {
-  CUtensorMap tmX, tmWg, tmW2, tmY;
-  RS_TRY(make_tmap(&tmX, x, C, M, 128));
-  RS_TRY(make_tmap(&tmWg, wg, C, H, 128));
-  RS_TRY(make_tmap(&tmW2, W2, H, C, rs::fused_w2_rows(C)));
-  RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
-  rs::FusedParams p{};
-  p.M = M;
-  p.C = C;
-  p.H = H;
-  p.num_m = (M + 127) / 128;
-  p.stats = reinterpret_cast<const float2*>(stats);
-  p.colG = colg;
-  p.colC = colc;
-  p.b2 = static_cast<const __nv_bfloat16*>(b2);
-  p.x = static_cast<const __nv_bfloat16*>(x);
-  p.partials = partials;
-  p.err = st.err;
-  p.timeout_ns = rs::kDefaultTimeoutNs;
-  RS_CUDA(rs::launch_mlp_fused(tmX, tmWg, tmW2, tmY, p, st.num_sms, s, pdl));
   return RS_OK;
 }
 
@@ -433,27 +404,6 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   return RS_OK;
 }
 
-int rs_mlp_fused_supported(int C, int H) { return rs::fused_supported(C, H) ? 1 : 0; }
-
-int rs_mlp_fused(const void* x, const float* stats, const void* Wg, const float* colG,
-                 const float* colC, int M, int C, int H, const void* W2, const void* b2, void* y,
-                 float* partials, void* stream) {
-  RS_TRY(check_width(C));
-  RS_TRY(check_hidden(H));
-  RS_TRY(check_rows(M, C, H));
-  if (!rs::fused_supported(C, H)) return RS_ERR_SHAPE;
-  if (M == 0) return RS_OK;
-  if (!x || !stats || !Wg || !colG || !colC || !W2 || !b2 || !y || !partials) return RS_ERR_NULL;
-  if (!al16(x) || !al8(stats) || !al16(Wg) || !al16(colG) || !al16(colC) || !al16(W2) ||
-      !al16(b2) || !al16(y) || !al4(partials))
-    return RS_ERR_ALIGN;
-  std::lock_guard<std::mutex> lock(g_mu);
-  DevState* st = nullptr;
-  RS_TRY(dev_state(&st));
-  return run_fused_step(*st, x, stats, Wg, colG, colC, M, C, H, W2, b2, y, partials,
-                        static_cast<cudaStream_t>(stream), false);
-}
-
 int rs_gelu_apply(const float* z, float* out, int n, void* stream) {
   if (n < 0) return RS_ERR_SHAPE;
   if (n == 0) return RS_OK;
@@ -564,21 +514,8 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
   void* hidden = ws + w.hidden;
   void* y = ws + w.y;
   float* partials = reinterpret_cast<float*>(ws + w.partials);
-  if (rs::fused_supported(C, H)) {
-    // narrow blocks: LN prep, then fc1 + GELU + fc2 + shift in one kernel
-    float* stats = reinterpret_cast<float*>(ws + w.stats);
-    void* wg = ws + w.wg;
-    float* colg = reinterpret_cast<float*>(ws + w.colg);
-    float* colc = reinterpret_cast<float*>(ws + w.colc);
-    RS_CUDA(rs::launch_ln_prep(x, M, C, stats, W1, gamma, beta, b1, H, wg, colg, colc,
-                               st->num_sms, s));
-    RS_TRY(run_fused_step(*st, x, stats, wg, colg, colc, M, C, H, W2, b2, y, partials, s,
-                          /*pdl=*/true));
-    RS_CUDA(rs::launch_select_gather(partials, rs::kFusedPartials, y, B, L, C, keep_k, scores,
-                                     kept_idx, y_kept, st->num_sms, s, /*pdl=*/true));
-    return RS_OK;
-  }
   const int np = rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
+
   RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
   RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s, /*pdl=*/true));
   RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, scores, kept_idx, y_kept,

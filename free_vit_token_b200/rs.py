@@ -38,8 +38,6 @@ SIGNATURES = {
     "rs_ln_fc1_gelu_noalloc": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_num_partials": (_i, [_i]),
-    "rs_mlp_fused_supported": (_i, [_i, _i]),
-    "rs_mlp_fused": (_i, [_vp, _fp, _vp, _fp, _fp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
     "rs_select_gather": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
@@ -227,31 +225,6 @@ def rs_fc2_residual_shift(hidden: torch.Tensor, x2d: torch.Tensor, W2, b2,
     st = lib().rs_fc2_residual_shift(_ptr(hidden), _ptr(x2d), M, C, H, _ptr(W2), _ptr(b2), _ptr(y),
                                      _ptr(partials), _stream(stream))
     _check(st, "rs_fc2_residual_shift")
-    return y, partials
-
-
-RS_FUSED_PARTIALS = 4
-
-
-def rs_mlp_fused_supported(C: int, H: int) -> bool:
-    return bool(lib().rs_mlp_fused_supported(int(C), int(H)))
-
-
-def rs_mlp_fused(x2d: torch.Tensor, stats: torch.Tensor, Wg: torch.Tensor, colG: torch.Tensor,
-                 colC: torch.Tensor, W2, b2, y: Optional[torch.Tensor] = None,
-                 partials: Optional[torch.Tensor] = None, stream=None
-                 ) -> Tuple[torch.Tensor, torch.Tensor]:
-    """The fused MLP on LN statistics and folded weights: (y [M, C] bf16,
-    partials [M, RS_FUSED_PARTIALS] fp32)."""
-    M, C = x2d.shape
-    H = Wg.shape[0]
-    if y is None:
-        y = torch.empty(M, C, dtype=torch.bfloat16, device=x2d.device)
-    if partials is None:
-        partials = torch.empty(M, RS_FUSED_PARTIALS, dtype=torch.float32, device=x2d.device)
-    st = lib().rs_mlp_fused(_ptr(x2d), _ptr(stats), _ptr(Wg), _ptr(colG), _ptr(colC), M, C, H,
-                            _ptr(W2), _ptr(b2), _ptr(y), _ptr(partials), _stream(stream))
-    _check(st, "rs_mlp_fused")
     return y, partials
 
 

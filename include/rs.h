@@ -78,11 +78,6 @@ typedef enum rs_status {
  *   y_kept   [B, 1+keep_k, C] bf16   output
  *   kept_idx [B, 1+keep_k] int32     output (4-byte aligned)
  *   scores   [B, L] fp32             output, every token incl. CLS (4-byte aligned)
- *
- * Kernels: LN statistics + weight fold, then for rs_mlp_fused_supported(C, H)
- * the fused MLP kernel (rs_mlp_fused), otherwise fc1 and fc2 as two GEMMs
- * (rs_fc1_gelu_folded, rs_fc2_residual_shift), then selection + gather
- * (rs_select_gather). The results are the same up to fp32 summation order.
  */
 int rs_block_forward(const void* x, int B, int L, int C, int H,
                      const void* W1, const void* b1, const void* W2, const void* b2,
@@ -142,25 +137,6 @@ int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H
 /* Number of per-row partial sums rs_fc2_residual_shift writes for width C
  * (0 if C is unsupported). */
 int rs_num_partials(int C);
-
-/* The MLP sublayer (§3.3 Eq. (6)) with the shift partials (Eq. (4)) in one
- * kernel, for narrow blocks: fc1 with the folded LayerNorm and GELU, fc2 with
- * b2 and the residual, the hidden activation kept in shared memory and never
- * stored. Inputs as for rs_fc1_gelu_folded (stats from rs_ln_stats; Wg, colG,
- * colC from rs_ln_fold) plus W2 [C, H] and b2 [C] bf16:
- *   a = bf16(GELU(rstd*(x' Wg^T - mean*G) + cb)), h = a W2^T + b2 (fp32),
- *   y = bf16(x' + h)  [M, C] bf16 output,
- *   partials[r, j] = sum over column quarter j (columns jC/4 .. (j+1)C/4-1) of
- *                    (h[r,c] - x'[r,c])^2, [M, RS_FUSED_PARTIALS] fp32 output
- *                    (4-byte aligned); summed left to right they give s_t^2.
- * rs_mlp_fused_supported(C, H) is 1 when 64 <= C <= 384 and H is a multiple of
- * 128, else 0; rs_mlp_fused returns RS_ERR_SHAPE outside that range. It uses no
- * workspace. rs_block_forward takes this path whenever it is supported. */
-#define RS_FUSED_PARTIALS 4
-int rs_mlp_fused_supported(int C, int H);
-int rs_mlp_fused(const void* x, const float* stats, const void* Wg, const float* colG,
-                 const float* colC, int M, int C, int H, const void* W2, const void* b2, void* y,
-                 float* partials, void* stream);
 
 /* Score finalisation and per-sample top-k (§3.2 drop the lowest-k scores):
  *   scores[b, t] = sqrt(sum_{j=0..P-1} partials[b*L+t, j])  (fp32, left to right)

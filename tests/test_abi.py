@@ -87,27 +87,6 @@ def test_step_entry_points_argument_errors():
     assert L.rs_gather_rows(FAKE, 2, 10, 192, None, 3, FAKE, None) == rs.RS_ERR_NULL
 
 
-def test_fused_entry_point_support_and_argument_errors():
-    L = rs.lib()
-    for C, H in [(384, 1536), (192, 768), (64, 128), (320, 640)]:
-        assert L.rs_mlp_fused_supported(C, H) == 1
-    for C, H in [(448, 1792), (768, 3072), (384, 1600), (384, 64), (100, 256)]:
-        assert L.rs_mlp_fused_supported(C, H) == 0
-
-    def f(x=FAKE, st=FAKE, M=10, C=384, H=1536, y=FAKE, parts=FAKE):
-        return L.rs_mlp_fused(x, st, FAKE, FAKE, FAKE, M, C, H, FAKE, FAKE, y, parts, None)
-
-    assert f(C=448, H=1792) == rs.RS_ERR_SHAPE
-    assert f(H=1600) == rs.RS_ERR_SHAPE
-    assert f(C=100) == rs.RS_ERR_SHAPE
-    assert f(M=0) == rs.RS_OK
-    assert f(x=None) == rs.RS_ERR_NULL
-    assert f(parts=None) == rs.RS_ERR_NULL
-    assert f(x=MIS) == rs.RS_ERR_ALIGN
-    assert f(st=FAKE + 4) == rs.RS_ERR_ALIGN  # stats are (mean, rstd) pairs: 8-byte aligned
-    assert f(parts=FAKE + 2) == rs.RS_ERR_ALIGN
-
-
 def test_library_has_no_torch_or_libcuda_link_dependency():
     out = os.popen(f"ldd {rs.LIB_PATH}").read()
     assert "libtorch" not in out and "libc10" not in out
