@@ -256,11 +256,13 @@ def main():
         flush_w.zero_()
         flush_r.sum()
 
-    def step(x0):
+    def step(x0, last=None):
+        """One pass of the block (every stage); `last` replaces the last stage's outputs."""
         xs = x0
         for s, k in enumerate(wl.keep_k):
-            rs.rs_block_forward(xs, *W[s], k, *outs[s], stream=stream)
-            xs = outs[s][0]
+            o = last if (last is not None and s == wl.stages - 1) else outs[s]
+            rs.rs_block_forward(xs, *W[s], k, *o, stream=stream)
+            xs = o[0]
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -344,6 +346,7 @@ def main():
     # graph and replayed (launch overhead amortised). y and the partials are the
     # ones fc2 just wrote in the breakdown above, L2-resident as in the block.
     sel_ms = 0.0
+    sel_ms_flushed = 0.0
     cap_stream = torch.cuda.Stream(dev)
     for s, k in enumerate(wl.keep_k):
         L_s = wl.stage_L(s)
@@ -368,6 +371,29 @@ def main():
             reps.append(a.elapsed_time(b) / SG_REPS)
         sel_ms += statistics.median(reps)
         del g
+        # the same launch right after an L2 flush: graph [flush, select+gather] minus [flush]
+        gf, gfs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf, stream=cap_stream):
+            flush_w.zero_()
+            flush_r.sum()
+        with torch.cuda.graph(gfs, stream=cap_stream):
+            flush_w.zero_()
+            flush_r.sum()
+            rs.rs_select_gather(p2, y2, k, scores=outs[s][2], kept_idx=outs[s][1],
+                                y_kept=outs[s][0], stream=cap_stream)
+        diffs = []
+        for _ in range(7):
+            tt = []
+            for g_ in (gf, gfs):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g_.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                tt.append(a.elapsed_time(b))
+            diffs.append(tt[1] - tt[0])
+        sel_ms_flushed += max(statistics.median(diffs), 1e-6)
+        del gf, gfs
     sg_bytes = 0
     for s, k in enumerate(wl.keep_k):
         M = wl.tokens(s)
@@ -376,28 +402,53 @@ def main():
     sg_gbs = sg_bytes / (sel_ms / 1e3) / 1e9
     block_flops = sum(4.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages))
 
-    # ---- end to end through the public call with host buffers
+    # ---- end to end through the public call with host buffers: every step copies its
+    # input x' from pinned host memory and its outputs (y_kept, kept_idx, scores) back to
+    # pinned host memory. Steps are pipelined as a serving loop would run them: the H2D
+    # copy of step i+1 and the D2H copy of step i-1 run on their own streams while step i
+    # computes (two device buffers for the input and for the outputs).
     x_h = inp.x.pin_memory()
     h2d = x_h.numel() * x_h.element_size()
-    outs_h = [tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs[-1])]
-    d2h = sum(o.numel() * o.element_size() for o in outs_h[0])
-    x_d = torch.empty_like(x)
+    outs_h = tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs[-1])
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+    x_d = [torch.empty_like(x) for _ in range(2)]
+    outs_d = [tuple(torch.empty_like(o) for o in outs[-1]) for _ in range(2)]
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     n_e2e = max(5, min(args.steps, 100))
-    e2e_ev = []
+    ev = lambda: torch.cuda.Event()
+    h2d_done, comp_done, d2h_done = [], [], []
     barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    s_h2d.wait_stream(stream)
+    s_d2h.wait_stream(stream)
     for i in range(n_e2e):
+        j = i & 1
+        if i >= 2:
+            s_h2d.wait_event(comp_done[i - 2])  # step i-2 has read x_d[j]
+        with torch.cuda.stream(s_h2d):
+            x_d[j].copy_(x_h, non_blocking=True)
+        h2d_done.append(ev())
+        h2d_done[-1].record(s_h2d)
+        stream.wait_event(h2d_done[i])
+        if i >= 2:
+            stream.wait_event(d2h_done[i - 2])  # outs_d[j] has reached the host
         l2_flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        x_d.copy_(x_h, non_blocking=True)
-        step(x_d)
-        for oh, od in zip(outs_h[0], outs[-1]):
-            oh.copy_(od, non_blocking=True)
-        b.record(stream)
-        e2e_ev.append((a, b))
+        step(x_d[j], last=outs_d[j])
+        comp_done.append(ev())
+        comp_done[-1].record(stream)
+        s_d2h.wait_event(comp_done[i])
+        with torch.cuda.stream(s_d2h):
+            for oh, od in zip(outs_h, outs_d[j]):
+                oh.copy_(od, non_blocking=True)
+        d2h_done.append(ev())
+        d2h_done[-1].record(s_d2h)
+    stream.wait_event(d2h_done[-1])
+    t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev) / n_e2e
+    e2e_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev) / n_e2e
     e2e_value = job_throughput(tokens_per_step, 1, e2e_ms, world)
     clocks.stop()
 
@@ -428,10 +479,17 @@ def main():
                           "bytes": sg_bytes, "ms": sel_ms,
                           "timing": f"device time per launch, {SG_REPS} launches replayed from a "
                                     "CUDA graph, inputs as fc2 left them (L2-resident)",
-                          "ms_single_launch_events": sel_ms_event},
+                          "ms_single_launch_events": sel_ms_event,
+                          "after_l2_flush": {"ms": sel_ms_flushed,
+                                             "GBps": sg_bytes / (sel_ms_flushed / 1e3) / 1e9,
+                                             "frac_hbm": sg_bytes / (sel_ms_flushed / 1e3) / 1e9
+                                             / peaks["hbm"],
+                                             "timing": "graph [256 MiB flush, select+gather] "
+                                                       "minus graph [flush], per launch"}},
         "images_per_s": world * wl.B / (ms_per_step / 1e3),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (own streams)"},
         "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
