@@ -123,16 +123,18 @@ struct SelSmem {
   uint32_t* warp;  // [33] block scan scratch
   uint32_t* hist;  // [256] radix histogram
   uint32_t* sel;   // [2] selected digit, count above it
+  uint32_t* rng;   // [2 * 32] per warp: smallest and largest patch key it loaded
 };
 
 __device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, uint32_t* s_hist,
-                                         uint32_t* s_sel) {
+                                         uint32_t* s_sel, uint32_t* s_rng) {
   SelSmem s;
   s.key = reinterpret_cast<uint32_t*>(dyn);
   s.kept = reinterpret_cast<int32_t*>(dyn + ((L + 3) & ~3) * 4);
   s.warp = s_warp;
   s.hist = s_hist;
   s.sel = s_sel;
+  s.rng = s_rng;
   return s;
 }
 
@@ -144,12 +146,52 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
   const int Lpad = (L + 3) & ~3;
   const int tid = threadIdx.x, nt = blockDim.x;
   const float* P = partials + static_cast<size_t>(b) * L * NP;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // over this thread's patch keys (t >= 1)
   auto finish = [&](int t, float acc) {
     const float v = sqrtf(acc);
     if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
-    s.key[t] = __float_as_uint(v);
+    const uint32_t key = __float_as_uint(v);
+    s.key[t] = key;
+    if (t >= 1) {
+      kmin = key < kmin ? key : kmin;
+      kmax = key > kmax ? key : kmax;
+    }
   };
-  if ((NP & 1) == 0 && NP <= 8) {
+  if ((NP & 3) == 0 && NP <= 8) {
+    // NP a multiple of 4: every row 16-byte aligned, one or two quad loads per row
+    const int np4 = NP >> 2;
+    const float4* P4 = reinterpret_cast<const float4*>(P);
+    for (int base = 0; base < Lpad; base += 4 * nt) {
+      float4 v[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = base + tid + i * nt;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          v[i][j] = (t < L && j < np4) ? __ldg(P4 + static_cast<size_t>(t) * np4 + j)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = base + tid + i * nt;
+        if (t < L) {
+          float acc = 0.f;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (j < np4) {
+              acc += v[i][j].x;
+              acc += v[i][j].y;
+              acc += v[i][j].z;
+              acc += v[i][j].w;
+            }
+          }
+          finish(t, acc);
+        } else if (t < Lpad) {
+          s.key[t] = 0u;
+        }
+      }
+    }
+  } else if ((NP & 1) == 0 && NP <= 8) {
     // an even NP keeps every row 8-byte aligned: up to four pairs per row
     const int np2 = NP >> 1;
     const float2* P2 = reinterpret_cast<const float2*>(P);
@@ -193,6 +235,12 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
       }
     }
   }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if ((threadIdx.x & 31) == 0) {
+    s.rng[2 * (threadIdx.x >> 5)] = kmin;
+    s.rng[2 * (threadIdx.x >> 5) + 1] = kmax;
+  }
   __syncthreads();
 }
 
@@ -222,20 +270,44 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
   const int Lpad = (L + 3) & ~3;
   const uint4* key4 = reinterpret_cast<const uint4*>(s.key);
   uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
+  // Every patch key lies in [kmin, kmax] (as unsigned integers), so the leading bits
+  // on which kmin and kmax agree are those of every key: such digits are taken
+  // without a histogram pass (typically the top byte: sign and high exponent bits).
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int w = 0; w < (nt >> 5); ++w) {
+    kmin = s.rng[2 * w] < kmin ? s.rng[2 * w] : kmin;
+    kmax = s.rng[2 * w + 1] > kmax ? s.rng[2 * w + 1] : kmax;
+  }
   for (int shift = 24; shift >= 0; shift -= 8) {
+    if (kmin <= kmax && ((kmin ^ kmax) >> shift) == 0) {
+      prefix |= kmin & (0xFFu << shift);
+      mask |= 0xFFu << shift;
+      continue;  // every key has this digit: none above it, `need` unchanged
+    }
     for (int i = tid; i < 256; i += nt) s.hist[i] = 0;
     __syncthreads();
     for (int base = 0; base < L; base += 4 * nt) {
       const int t0 = base + 4 * tid;
       const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
       const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+      if (shift == 24) {
+        // top byte (sign and high exponent bits): few distinct values, so lanes with
+        // the same digit are aggregated into one atomic
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = t0 + i;
-        const bool cand = t >= 1 && t < L && (u[i] & mask) == prefix;
-        const uint32_t digit = cand ? ((u[i] >> shift) & 0xFFu) : 256u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + i;
+          const bool cand = t >= 1 && t < L;
+          const uint32_t digit = cand ? (u[i] >> 24) : 256u;
+          const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+          if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
+        }
+      } else {
+        // lower digits are spread out: one atomic per candidate key
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + i;
+          if (t >= 1 && t < L && (u[i] & mask) == prefix) atomicAdd(&s.hist[(u[i] >> shift) & 0xFFu], 1u);
+        }
       }
     }
     __syncthreads();
@@ -313,11 +385,11 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
                                                       int L, int k, float* __restrict__ scores,
                                                       int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2];
+  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
-  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel);
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
   load_keys(partials, NP, L, b, scores, s);
   select_into_smem(L, k, s);
   int32_t* out = kept + static_cast<size_t>(b) * (k + 1);
@@ -376,12 +448,12 @@ __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_ga
     const float* __restrict__ partials, int NP, int L, int k, const uint4* __restrict__ y, int Cv,
     int S, float* __restrict__ scores, int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2];
+  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x / S, j0 = blockIdx.x % S;
   const bool writer = j0 == 0;
-  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel);
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
   load_keys(partials, NP, L, b, writer ? scores : nullptr, s);
   select_into_smem(L, k, s);
   const int k1 = k + 1;
