@@ -16,7 +16,8 @@ output), written out literally and in float64 throughout:
 4. s_t = || MLP(LN(x'_t)) - x'_t ||_2 -- the representation shift of Eq. (4) with
                                        F = the MLP (§3.3 "Operation choice", case
                                        (ii)) and D = the L2 distance (§3.3
-                                       "Distance metrics", case (i))
+                                       "Distance metrics", case (i)); the L1 and
+                                       cosine distances (cases (ii), (iii)) too
 5. drop the lowest-s patch tokens, keep CLS plus the k highest (§3.1 pruned set
    x-tilde in R^{(N-r) x C}; §3.2 "dropped the tokens having the lowest k scores")
 6. gather the kept rows of y.
@@ -27,6 +28,8 @@ Readings where the pages are silent (each also listed in the design notes):
 * The score compares the MLP output *without* the residual against x' (Eq. (4)
   with F = MLP o LN as §3.3 writes it), i.e. h - x', not y - x'.
 * CLS (t = 0) is always kept and never ranked; its score is still reported.
+  Without a CLS token (cls=False) all L tokens are ranked.
+* The cosine distance floors ||h|| ||x'|| at 1e-8; in fp32 it is floored at 0.
 * Ties in s go to the lower token index; kept rows are in ascending index order.
 
 Pins (tests/test_oracle_pins.py): a hand-worked 4-token example checked against
@@ -67,33 +70,54 @@ def mlp(u: np.ndarray, W1, b1, W2, b2) -> np.ndarray:
     return fc(gelu(fc(u, W1, b1)), W2, b2)
 
 
-def shift_score(h: np.ndarray, x: np.ndarray) -> np.ndarray:
-    """Representation shift, Eq. (4) with D = L2 (§3.2): ||F(x) - x||_2 per row."""
-    return np.sqrt(((h - x) ** 2).sum(axis=-1))
+METRICS = ("l2", "l1", "cosine")
+COS_EPS = 1e-8  # floor of ||h|| ||x|| in the cosine distance (the pages give none)
 
 
-def sublayer(x: np.ndarray, W1, b1, W2, b2, gamma, beta, eps: float = EPS):
+def shift_score(h: np.ndarray, x: np.ndarray, metric: str = "l2") -> np.ndarray:
+    """Representation shift, Eq. (4), D(F(x'), x') per row with F(x') = h, the MLP output
+    (§3.3 "Operation choice" (ii)) and D one of §3.3 "Distance metrics":
+      (i)   l2:     ||h - x||_2
+      (ii)  l1:     ||h - x||_1
+      (iii) cosine: 1 - h.x / (||h|| ||x||), the denominator floored at COS_EPS.
+    """
+    if metric == "l2":
+        return np.sqrt(((h - x) ** 2).sum(axis=-1))
+    if metric == "l1":
+        return np.abs(h - x).sum(axis=-1)
+    if metric == "cosine":
+        dot = (h * x).sum(axis=-1)
+        den = np.sqrt((h * h).sum(axis=-1)) * np.sqrt((x * x).sum(axis=-1))
+        return 1.0 - dot / np.maximum(den, COS_EPS)
+    raise ValueError(f"unknown metric {metric!r}")
+
+
+def sublayer(x: np.ndarray, W1, b1, W2, b2, gamma, beta, eps: float = EPS, metric: str = "l2"):
     """Eq. (6) for token rows x = x' [..., C]: returns (h, y, s)."""
     h = mlp(layer_norm(x, gamma, beta, eps), W1, b1, W2, b2)
     y = h + x
-    s = shift_score(h, x)
+    s = shift_score(h, x, metric)
     return h, y, s
 
 
-def select_topk(s: np.ndarray, k: int) -> np.ndarray:
-    """Kept token indices for one sample: [0] ++ ascending(top-k patch tokens by s).
+def select_topk(s: np.ndarray, k: int, cls: bool = True) -> np.ndarray:
+    """Kept token indices for one sample.
 
-    Patch tokens are t = 1..L-1. They are ordered by decreasing s, equal s by
-    increasing t (a stable sort), and the first k are kept. CLS (t = 0) is
-    always first and never ranked.
+    With a CLS token (cls=True): [0] ++ ascending(top-k patch tokens by s); patch
+    tokens are t = 1..L-1 and CLS (t = 0) is always first and never ranked.
+    Without (cls=False, a video sequence of patch tokens only): ascending(top-k of all
+    L tokens). Ranking: decreasing s, equal s by increasing t (a stable sort).
     """
     L = s.shape[0]
-    if not 0 <= k <= L - 1:
+    first = 1 if cls else 0
+    if not 0 <= k <= L - first:
         raise ValueError("keep_k out of range")
-    t = np.arange(1, L)
-    order = np.lexsort((t, -s[1:]))  # primary key -s, secondary key t
-    kept = np.sort(t[order[:k]])
-    return np.concatenate([np.zeros(1, dtype=np.int64), kept]).astype(np.int64)
+    t = np.arange(first, L)
+    order = np.lexsort((t, -s[first:]))  # primary key -s, secondary key t
+    kept = np.sort(t[order[:k]]).astype(np.int64)
+    if cls:
+        return np.concatenate([np.zeros(1, dtype=np.int64), kept])
+    return kept
 
 
 def gather(y: np.ndarray, kept: np.ndarray) -> np.ndarray:
@@ -101,30 +125,53 @@ def gather(y: np.ndarray, kept: np.ndarray) -> np.ndarray:
     return y[kept]
 
 
-def block_forward(x, W1, b1, W2, b2, gamma, beta, keep_k: int, eps: float = EPS):
+def block_forward(x, W1, b1, W2, b2, gamma, beta, keep_k: int, eps: float = EPS,
+                  metric: str = "l2", cls: bool = True):
     """The whole path for x [B, L, C] (float64 values of the stored inputs).
 
-    Returns (y_kept [B, 1+k, C], kept_idx [B, 1+k], scores [B, L], y [B, L, C]).
+    Returns (y_kept [B, n, C], kept_idx [B, n], scores [B, L], y [B, L, C]) with
+    n = 1 + k (CLS kept) or k (cls=False).
     """
     x = np.asarray(x, dtype=np.float64)
     B, L, C = x.shape
-    _, y, s = sublayer(x.reshape(B * L, C), W1, b1, W2, b2, gamma, beta, eps)
+    _, y, s = sublayer(x.reshape(B * L, C), W1, b1, W2, b2, gamma, beta, eps, metric)
     y = y.reshape(B, L, C)
     s = s.reshape(B, L)
-    kept = np.stack([select_topk(s[b], keep_k) for b in range(B)])
+    kept = np.stack([select_topk(s[b], keep_k, cls) for b in range(B)])
     y_kept = np.stack([gather(y[b], kept[b]) for b in range(B)])
     return y_kept, kept, s, y
 
 
-def finalize_scores_f32(partials: np.ndarray, B: int, L: int) -> np.ndarray:
-    """Scores from fp32 per-row partial sums of squares, in fp32.
+def finalize_scores_f32(partials: np.ndarray, B: int, L: int, metric: str = "l2") -> np.ndarray:
+    """Scores from fp32 per-row partial sums, in fp32 (correctly rounded operations).
 
-    s = sqrt(sum_j P[r, j]) with the partials added left to right in fp32 and a
-    correctly rounded fp32 square root. Used where an fp32 score decides the
-    integer kept set, so that both sides rank the same fp32 keys.
+    l2:     partials are sums of (h - x)^2 over column groups; s = sqrt(sum_j P[r, j]).
+    l1:     partials are sums of |h - x|; s = sum_j P[r, j].
+    cosine: partials are triples (sum h.x, sum h.h, sum x.x) per column group;
+            s = max(0, 1 - HX / max(sqrt(HH) * sqrt(XX), COS_EPS)) with HX, HH, XX the
+            group sums. Floored at 0 so that the fp32 bits order like the values.
+    Partials are added left to right (group order). Used where an fp32 score decides
+    the integer kept set, so that both sides rank the same fp32 keys.
     """
-    p = np.asarray(partials, dtype=np.float32).reshape(B * L, -1)
-    acc = np.zeros(B * L, dtype=np.float32)
-    for j in range(p.shape[1]):
-        acc = (acc + p[:, j]).astype(np.float32)
-    return np.sqrt(acc).astype(np.float32).reshape(B, L)
+    f32 = np.float32
+    p = np.asarray(partials, dtype=f32).reshape(B * L, -1)
+
+    def rsum(cols):
+        acc = np.zeros(B * L, dtype=f32)
+        for j in cols:
+            acc = (acc + p[:, j]).astype(f32)
+        return acc
+
+    if metric == "l2":
+        return np.sqrt(rsum(range(p.shape[1]))).astype(f32).reshape(B, L)
+    if metric == "l1":
+        return rsum(range(p.shape[1])).reshape(B, L)
+    if metric == "cosine":
+        if p.shape[1] % 3:
+            raise ValueError("cosine partials come in triples")
+        n = p.shape[1]
+        hx, hh, xx = rsum(range(0, n, 3)), rsum(range(1, n, 3)), rsum(range(2, n, 3))
+        den = np.maximum((np.sqrt(hh) * np.sqrt(xx)).astype(f32), f32(COS_EPS))
+        s = (f32(1.0) - (hx / den).astype(f32)).astype(f32)
+        return np.maximum(s, f32(0.0)).reshape(B, L)
+    raise ValueError(f"unknown metric {metric!r}")

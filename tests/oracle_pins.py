@@ -121,9 +121,10 @@ def pin_first_layer_zero(o):
 
 def pin_loops(o):
     """LayerNorm, fc1, fc2, the residual and the score, index by index."""
-    rng = np.random.default_rng(13)
-    for C, H, L in ((3, 5, 4), (4, 4, 3)):  # the square case catches a transposed weight
-        _loops_case(o, rng, C, H, L)
+    # the square case first: a transposed weight then fails an assertion rather than
+    # a shape check
+    for seed, (C, H, L) in ((14, (4, 4, 3)), (13, (3, 5, 4))):
+        _loops_case(o, np.random.default_rng(seed), C, H, L)
 
 
 def _loops_case(o, rng, C, H, L):
@@ -152,11 +153,11 @@ def pin_ln_moments(o):
     assert np.abs((u ** 2).mean(axis=1) - 1.0).max() < 1e-12
 
 
-def _unique_topk_by_dominance(s, k):
-    """All k-subsets S of 1..L-1 such that every kept token beats every dropped one
+def _unique_topk_by_dominance(s, k, first=1):
+    """All k-subsets S of first..L-1 such that every kept token beats every dropped one
     (larger s, or equal s and lower index). Exactly one exists."""
     L = len(s)
-    pats = range(1, L)
+    pats = range(first, L)
     out = []
     for S in itertools.combinations(pats, k):
         Sset = set(S)
@@ -221,6 +222,124 @@ def pin_cls_kept(o):
         assert len(kept[0]) == 1 + k
 
 
+def pin_metrics_hand_example(o):
+    """L1 and cosine distances (§3.3 "Distance metrics" (ii), (iii)) on the 4-token
+    identity-weight case, by hand from Phi(1): every row has h = [P, -Q, P, -Q] with
+    P = Phi(1), Q = Phi(-1) = 1 - P, so h - x and h.x follow row by row. The kept sets
+    differ by metric (cosine ranks t1, t3 above t2), and without a CLS token t0 competes."""
+    g = _golden("hand_example_4tok.json")
+    P = _golden("normal_cdf_table.json")["phi"]["1.0"]
+    Q = 1.0 - P
+    x = np.array(g["x"], dtype=np.float64)
+    w = _identity_weights(4)
+    nh = math.sqrt(2 * (P * P + Q * Q))
+    l1 = [2 + 4 * Q, 2.0, 6 + 4 * Q, 2.0]
+    cos = [1 - 4 * P / (math.sqrt(8) * nh), 1 - 1 / nh,
+           1 - (6 * P - 2 * Q) / (math.sqrt(20) * nh), 1 - 1 / nh]
+    _, _, s1 = o.sublayer(x, eps=0.0, metric="l1", **w)
+    assert np.allclose(s1, l1, rtol=0, atol=1e-12), (s1, l1)
+    _, _, sc = o.sublayer(x, eps=0.0, metric="cosine", **w)
+    assert np.allclose(sc, cos, rtol=0, atol=1e-12), (sc, cos)
+    expect = {
+        ("l1", True): {0: [0], 1: [0, 2], 2: [0, 1, 2], 3: [0, 1, 2, 3]},
+        ("cosine", True): {0: [0], 1: [0, 1], 2: [0, 1, 3], 3: [0, 1, 2, 3]},
+        # no CLS: L2 scores 1.65, 1.21, 3.46, 1.21 rank t2, t0, then the tied t1, t3
+        ("l2", False): {0: [], 1: [2], 2: [0, 2], 3: [0, 1, 2], 4: [0, 1, 2, 3]},
+        ("cosine", False): {0: [], 1: [1], 2: [1, 3], 3: [1, 2, 3], 4: [0, 1, 2, 3]},
+    }
+    for (metric, cls), kept_by_k in expect.items():
+        for k, kept in kept_by_k.items():
+            yk, kidx, sc_, _ = o.block_forward(x[None], keep_k=k, eps=0.0, metric=metric,
+                                               cls=cls, **w)
+            assert list(kidx[0]) == kept, (metric, cls, k, list(kidx[0]), kept)
+            assert yk.shape == (1, len(kept), 4)
+
+
+def pin_metric_invariants(o):
+    """Norm inequalities between L1 and L2, the range of the cosine distance, its
+    indifference to the length of h, and parallel / antiparallel / orthogonal cases."""
+    rng = np.random.default_rng(19)
+    C = 16
+    h = rng.normal(0, 1, (6, C))
+    x = rng.normal(0, 1, (6, C))
+    l2, l1, cs = (o.shift_score(h, x, m) for m in ("l2", "l1", "cosine"))
+    assert np.all(l1 >= l2 - 1e-12) and np.all(l1 <= math.sqrt(C) * l2 + 1e-12)
+    assert np.all(cs >= 0) and np.all(cs <= 2)
+    # scaling h by 2 is exact in binary floating point: the cosine distance is unchanged
+    # bit for bit, while L1 and L2 are not
+    assert np.array_equal(o.shift_score(2 * h, x, "cosine"), cs)
+    assert not np.allclose(o.shift_score(2 * h, x, "l2"), l2)
+    v = x[:1]
+    assert abs(o.shift_score(v, v, "cosine")[0]) < 1e-15
+    assert abs(o.shift_score(-v, v, "cosine")[0] - 2.0) < 1e-15
+    e = np.eye(C)
+    assert o.shift_score(e[:1], e[1:2], "cosine")[0] == 1.0
+    d = np.zeros((1, C))
+    d[0, 3] = -2.5
+    assert o.shift_score(x[:1] + d, x[:1], "l1")[0] == 2.5
+    assert o.shift_score(x[:1] + d, x[:1], "l2")[0] == 2.5
+
+
+def pin_topk_no_cls_exhaustive(o):
+    """Without a CLS token: kept set = the unique dominance-closed k-subset of all L
+    tokens, for every k, with ties."""
+    rng = np.random.default_rng(20)
+    for L in (1, 2, 5, 8, 10):
+        for trial in range(3):
+            s = rng.integers(0, 4, L).astype(np.float64) * 0.5
+            if trial == 2:
+                s = rng.random(L)
+            for k in range(0, L + 1):
+                sols = _unique_topk_by_dominance(s, k, first=0)
+                assert len(sols) == 1
+                got = o.select_topk(s, k, cls=False)
+                assert list(got) == list(sols[0]), (L, k, s, got, sols)
+
+
+def pin_permutation_no_cls(o):
+    """Without a CLS token, permuting all rows (t0 included) permutes the scores and maps
+    the kept set."""
+    rng = np.random.default_rng(21)
+    C, H, L, k = 8, 16, 11, 4
+    w = _rng_weights(rng, C, H)
+    x = rng.normal(0, 1, (1, L, C))
+    perm = rng.permutation(L)
+    for metric in ("l2", "cosine"):
+        yk, kept, s, y = o.block_forward(x, keep_k=k, metric=metric, cls=False, **w)
+        yk2, kept2, s2, y2 = o.block_forward(x[:, perm], keep_k=k, metric=metric, cls=False, **w)
+        assert np.array_equal(s2[0], s[0][perm])
+        assert len(set(s[0])) == L
+        assert sorted(perm[kept2[0]]) == sorted(kept[0]) and len(kept[0]) == k
+        assert np.all(np.diff(kept2[0]) > 0)
+        assert np.array_equal(yk2[0], y2[0][kept2[0]])
+
+
+def pin_finalize_f32(o):
+    """fp32 score finalisation of each metric on exactly representable cases, and against
+    its fp64 definition on random partials within fp32 rounding."""
+    f = o.finalize_scores_f32
+    assert f(np.array([[9.0, 16.0]]), 1, 1, "l2")[0, 0] == 5.0
+    assert f(np.array([[0.5, 0.25, 1.0]]), 1, 1, "l1")[0, 0] == 1.75
+    tri = np.array([[4.0, 4.0, 4.0],      # parallel: 1 - 4 / (2 * 2) = 0
+                    [0.0, 4.0, 9.0],      # orthogonal: 1
+                    [-6.0, 4.0, 9.0],     # antiparallel: 1 + 6 / 6 = 2
+                    [4.0, 2.0, 8.0],      # |h.x| above ||h|| ||x||: floored at 0
+                    [0.0, 0.0, 9.0]])     # h = 0: 1 - 0 / 1e-8 = 1
+    got = f(tri, 1, 5, "cosine")[0]
+    assert list(got) == [0.0, 1.0, 2.0, 0.0, 1.0], got
+    # two column groups: the triples are summed component-wise first
+    two = np.array([[1.0, 1.0, 2.0, 1.0, 3.0, 2.0]])  # HX = 2, HH = 4, XX = 4
+    assert f(two, 1, 1, "cosine")[0, 0] == 0.5
+    rng = np.random.default_rng(22)
+    p = rng.random((40, 6)).astype(np.float32)
+    p64 = p.astype(np.float64)
+    assert np.allclose(f(p, 1, 40, "l2")[0], np.sqrt(p64.sum(1)), rtol=1e-6)
+    assert np.allclose(f(p, 1, 40, "l1")[0], p64.sum(1), rtol=1e-6)
+    hx, hh, xx = p64[:, 0::3].sum(1), p64[:, 1::3].sum(1), p64[:, 2::3].sum(1)
+    ref = np.maximum(1 - hx / np.sqrt(hh * xx), 0)
+    assert np.allclose(f(p, 1, 40, "cosine")[0], ref, rtol=0, atol=1e-6)
+
+
 def pin_gather(o):
     """The kept rows of y, in kept order."""
     rng = np.random.default_rng(18)
@@ -231,6 +350,11 @@ def pin_gather(o):
 
 ALL_PINS = [
     pin_gelu_table,
+    pin_metrics_hand_example,
+    pin_metric_invariants,
+    pin_topk_no_cls_exhaustive,
+    pin_permutation_no_cls,
+    pin_finalize_f32,
     pin_hand_example,
     pin_zero_shift,
     pin_first_layer_zero,

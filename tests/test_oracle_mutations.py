@@ -12,7 +12,8 @@ import oracle.rs_oracle as rs_oracle
 from oracle_pins import ALL_PINS
 
 orig = {n: getattr(rs_oracle, n) for n in
-        ["layer_norm", "gelu", "fc", "mlp", "shift_score", "select_topk", "gather", "sublayer"]}
+        ["layer_norm", "gelu", "fc", "mlp", "shift_score", "select_topk", "gather", "sublayer",
+         "finalize_scores_f32"]}
 
 
 def _ln_unbiased(x, gamma, beta, eps=rs_oracle.EPS):
@@ -57,6 +58,20 @@ def _mlp_no_act(u, W1, b1, W2, b2):
     return rs_oracle.fc(rs_oracle.fc(u, W1, b1), W2, b2)
 
 
+# Mutants of one metric (or of the CLS mode) delegate every other case to the
+# original function, so that a pin has to catch the planted mistake itself.
+def _for_metric(metric, bad):
+    def f(h, x, m="l2"):
+        return bad(h, x) if m == metric else orig["shift_score"](h, x, m)
+    return f
+
+
+def _for_cls(bad):
+    def f(s, k, cls=True):
+        return bad(s, k) if cls else orig["select_topk"](s, k, cls)
+    return f
+
+
 def _score_plus(h, x):
     return np.sqrt(((h + x) ** 2).sum(axis=-1))
 
@@ -71,6 +86,23 @@ def _score_squared(h, x):
 
 def _score_l1(h, x):
     return np.abs(h - x).sum(axis=-1)
+
+
+def _l1_no_abs(h, x):
+    return (h - x).sum(axis=-1)
+
+
+def _cos_similarity(h, x):  # the similarity, not the distance
+    return (h * x).sum(-1) / (np.linalg.norm(h, axis=-1) * np.linalg.norm(x, axis=-1))
+
+
+def _cos_of_output(h, x):  # angle between y = h + x and x
+    y = h + x
+    return 1 - (y * x).sum(-1) / (np.linalg.norm(y, axis=-1) * np.linalg.norm(x, axis=-1))
+
+
+def _cos_unnormalised(h, x):
+    return 1 - (h * x).sum(-1)
 
 
 def _select_ties_high(s, k):
@@ -101,19 +133,46 @@ def _select_unsorted(s, k):
     return np.concatenate([[0], t[order[:k]]]).astype(np.int64)
 
 
+def _no_cls_still_keeps_cls(s, k, cls=True):
+    return orig["select_topk"](s, k, True) if not cls or True else None
+
+
+def _no_cls_skips_t0(s, k, cls=True):
+    if cls:
+        return orig["select_topk"](s, k, True)
+    if k > len(s) - 1:
+        k = len(s) - 1
+    return orig["select_topk"](s, k, True)[1:]
+
+
 def _gather_shift(y, kept):
     return y[np.minimum(kept + 1, y.shape[0] - 1)]
 
 
-def _sublayer_score_after_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS):
+def _sublayer_score_after_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS,
+                                   metric="l2"):
     h = rs_oracle.mlp(rs_oracle.layer_norm(x, gamma, beta, eps), W1, b1, W2, b2)
     y = h + x
-    return h, y, rs_oracle.shift_score(y, x)
+    return h, y, rs_oracle.shift_score(y, x, metric)
 
 
-def _sublayer_no_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS):
+def _sublayer_no_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS, metric="l2"):
     h = rs_oracle.mlp(rs_oracle.layer_norm(x, gamma, beta, eps), W1, b1, W2, b2)
-    return h, h, rs_oracle.shift_score(h, x)
+    return h, h, rs_oracle.shift_score(h, x, metric)
+
+
+def _finalize_cos_no_floor(partials, B, L, metric="l2"):
+    if metric != "cosine":
+        return orig["finalize_scores_f32"](partials, B, L, metric)
+    p = np.asarray(partials, dtype=np.float32).reshape(B * L, -1)
+    hx, hh, xx = (p[:, i::3].sum(1, dtype=np.float32) for i in range(3))
+    return (1 - hx / (np.sqrt(hh) * np.sqrt(xx) + np.float32(1e-8))).reshape(B, L)
+
+
+def _finalize_l1_sqrt(partials, B, L, metric="l2"):
+    if metric != "l1":
+        return orig["finalize_scores_f32"](partials, B, L, metric)
+    return orig["finalize_scores_f32"](partials, B, L, "l2")
 
 
 MUTATIONS = {
@@ -127,14 +186,23 @@ MUTATIONS = {
     "fc_drops_bias": ("fc", _fc_no_bias),
     "mlp_relu": ("mlp", _mlp_relu),
     "mlp_no_activation": ("mlp", _mlp_no_act),
-    "score_plus_sign": ("shift_score", _score_plus),
-    "score_squared": ("shift_score", _score_squared),
-    "score_l1": ("shift_score", _score_l1),
-    "score_of_h_only": ("shift_score", _score_residual),
-    "select_ties_to_higher_index": ("select_topk", _select_ties_high),
-    "select_keeps_lowest": ("select_topk", _select_lowest),
-    "select_ranks_cls": ("select_topk", _select_rank_cls),
-    "select_unsorted_output": ("select_topk", _select_unsorted),
+    "score_plus_sign": ("shift_score", _for_metric("l2", _score_plus)),
+    "score_squared": ("shift_score", _for_metric("l2", _score_squared)),
+    "score_l1": ("shift_score", _for_metric("l2", _score_l1)),
+    "score_of_h_only": ("shift_score", _for_metric("l2", _score_residual)),
+    "l1_squared": ("shift_score", _for_metric("l1", _score_squared)),
+    "l1_without_abs": ("shift_score", _for_metric("l1", _l1_no_abs)),
+    "cosine_similarity_not_distance": ("shift_score", _for_metric("cosine", _cos_similarity)),
+    "cosine_of_block_output": ("shift_score", _for_metric("cosine", _cos_of_output)),
+    "cosine_unnormalised": ("shift_score", _for_metric("cosine", _cos_unnormalised)),
+    "select_ties_to_higher_index": ("select_topk", _for_cls(_select_ties_high)),
+    "select_keeps_lowest": ("select_topk", _for_cls(_select_lowest)),
+    "select_ranks_cls": ("select_topk", _for_cls(_select_rank_cls)),
+    "select_unsorted_output": ("select_topk", _for_cls(_select_unsorted)),
+    "no_cls_still_keeps_cls": ("select_topk", _no_cls_still_keeps_cls),
+    "no_cls_never_keeps_t0": ("select_topk", _no_cls_skips_t0),
+    "finalize_cosine_not_floored": ("finalize_scores_f32", _finalize_cos_no_floor),
+    "finalize_l1_takes_sqrt": ("finalize_scores_f32", _finalize_l1_sqrt),
     "gather_off_by_one": ("gather", _gather_shift),
     "score_after_residual": ("sublayer", _sublayer_score_after_residual),
     "no_residual": ("sublayer", _sublayer_no_residual),
