@@ -4,6 +4,11 @@ The compute lives in ``librs.so`` (CUDA kernels behind a C ABI, include/rs.h);
 ``free_vit_token_b200.rs`` is its ctypes binding.
 """
 from .rs import (  # noqa: F401
+    DISTANCES,
+    RS_DIST_COSINE,
+    RS_DIST_L1,
+    RS_DIST_L2,
+    RS_NO_CLS,
     RsError,
     lib,
     rs_block_forward,

@@ -51,8 +51,9 @@ WsLayout ws_layout(int64_t M, int C, int H) {
   off = align_up(off + static_cast<size_t>(M) * H * 2, 1024);
   w.y = off;
   off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
-  w.partials = off;
-  off = align_up(off + static_cast<size_t>(M) * (rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C)) * 4,
+  w.partials = off;  // room for the cosine distance's three partials per column group
+  off = align_up(off + static_cast<size_t>(M) * rs::dist_partials(rs::kDistCos) *
+                           (rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C)) * 4,
                  1024);
   w.total = off;
   return w;
@@ -203,7 +204,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
 }
 
 int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H, const void* W2,
-            const void* b2, void* y, float* partials, cudaStream_t s, bool pdl = false) {
+            const void* b2, void* y, float* partials, int dist, cudaStream_t s, bool pdl = false) {
   const int bn = rs::fc2_block_n(C);
   const bool pair = rs::gemm_pair(M, H, false);
   CUtensorMap tmH, tmW, tmY;
@@ -220,11 +221,31 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.out = static_cast<__nv_bfloat16*>(y);
   p.resid = static_cast<const __nv_bfloat16*>(x);
   p.partials = partials;
-  p.num_partials = rs::kFc2PartialsPerTile * p.n_blocks;
+  p.dist = dist;
+  p.num_partials = rs::dist_partials(dist) * rs::kFc2PartialsPerTile * p.n_blocks;
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
   RS_CUDA(rs::launch_fc2(tmH, tmW, tmY, p, bn, pair, st.num_sms, s, pdl));
+  return RS_OK;
+}
+
+// The distance (RS_DIST_*) and the flags (RS_NO_CLS) of an extended entry point.
+int check_mode(int distance, int flags) {
+  if (distance != RS_DIST_L2 && distance != RS_DIST_L1 && distance != RS_DIST_COSINE)
+    return RS_ERR_SHAPE;
+  if ((flags & ~RS_NO_CLS) != 0) return RS_ERR_SHAPE;
+  return RS_OK;
+}
+// keep_k: 0..L-1 patch tokens with a CLS token, 0..L tokens without.
+int check_keep(int keep_k, int L, int flags) {
+  const int max_k = (flags & RS_NO_CLS) ? L : L - 1;
+  return (keep_k < 0 || keep_k > max_k) ? RS_ERR_KEEP_K : RS_OK;
+}
+// Partials per row: 1..64, and whole triples for the cosine distance.
+int check_partials(int num_partials, int distance) {
+  if (num_partials < 1 || num_partials > 64) return RS_ERR_SHAPE;
+  if (distance == RS_DIST_COSINE && num_partials % 3 != 0) return RS_ERR_SHAPE;
   return RS_OK;
 }
 
@@ -237,7 +258,8 @@ const char* rs_status_string(int status) {
     case RS_OK: return "RS_OK";
     case RS_ERR_NULL: return "RS_ERR_NULL: a required pointer is NULL";
     case RS_ERR_SHAPE: return "RS_ERR_SHAPE: B, L, C or H outside the supported limits";
-    case RS_ERR_KEEP_K: return "RS_ERR_KEEP_K: keep_k outside 0..L-1";
+    case RS_ERR_KEEP_K:
+      return "RS_ERR_KEEP_K: keep_k outside 0..L-1 (0..L without a CLS token)";
     case RS_ERR_ALIGN: return "RS_ERR_ALIGN: a pointer is not suitably aligned";
     case RS_ERR_CUDA: return "RS_ERR_CUDA: the CUDA runtime or driver reported an error";
     case RS_ERR_DEVICE_TIMEOUT: return "RS_ERR_DEVICE_TIMEOUT: a kernel pipeline wait timed out";
@@ -246,9 +268,11 @@ const char* rs_status_string(int status) {
   }
 }
 
-int rs_num_partials(int C) {
-  return check_width(C) == RS_OK ? rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C) : 0;
+int rs_num_partials_ex(int C, int distance) {
+  if (check_width(C) != RS_OK || check_mode(distance, 0) != RS_OK) return 0;
+  return rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
 }
+int rs_num_partials(int C) { return rs_num_partials_ex(C, RS_DIST_L2); }
 
 uint64_t rs_workspace_bytes(int B, int L, int C, int H) {
   if (B < 0 || L < 1 || check_width(C) != RS_OK || check_hidden(H) != RS_OK) return 0;
@@ -413,8 +437,10 @@ int rs_gelu_apply(const float* z, float* out, int n, void* stream) {
   return RS_OK;
 }
 
-int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H, const void* W2,
-                          const void* b2, void* y, float* partials, void* stream) {
+int rs_fc2_residual_shift_ex(const void* hidden, const void* x, int M, int C, int H,
+                             const void* W2, const void* b2, int distance, void* y,
+                             float* partials, void* stream) {
+  RS_TRY(check_mode(distance, 0));
   RS_TRY(check_width(C));
   RS_TRY(check_hidden(H));
   RS_TRY(check_rows(M, C, H));
@@ -425,33 +451,49 @@ int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H
   std::lock_guard<std::mutex> lock(g_mu);
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
-  return run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, static_cast<cudaStream_t>(stream));
+  return run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, distance,
+                 static_cast<cudaStream_t>(stream));
+}
+int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H, const void* W2,
+                          const void* b2, void* y, float* partials, void* stream) {
+  return rs_fc2_residual_shift_ex(hidden, x, M, C, H, W2, b2, RS_DIST_L2, y, partials, stream);
 }
 
-int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
-                   float* scores, int32_t* kept_idx, void* stream) {
-  if (B < 0 || L < 1 || L > RS_MAX_L || num_partials < 1 || num_partials > 64)
-    return RS_ERR_SHAPE;
+int rs_select_topk_ex(const float* partials, int num_partials, int B, int L, int keep_k,
+                      int distance, int flags, float* scores, int32_t* kept_idx, void* stream) {
+  RS_TRY(check_mode(distance, flags));
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_partials(num_partials, distance));
   if (static_cast<int64_t>(B) * L * num_partials >= (static_cast<int64_t>(1) << 31))
     return RS_ERR_SHAPE;
-  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  RS_TRY(check_keep(keep_k, L, flags));
   if (B == 0) return RS_OK;
-  if (!partials || !scores || !kept_idx) return RS_ERR_NULL;
+  if (!partials || !scores || (!kept_idx && keep_k + !(flags & RS_NO_CLS) > 0)) return RS_ERR_NULL;
   if (!al4(partials) || !al4(scores) || !al4(kept_idx)) return RS_ERR_ALIGN;
-  RS_CUDA(rs::launch_select(partials, num_partials, B, L, keep_k, scores, kept_idx,
+  RS_CUDA(rs::launch_select(partials, num_partials, B, L, keep_k, distance,
+                            !(flags & RS_NO_CLS), scores, kept_idx,
                             static_cast<cudaStream_t>(stream)));
   return RS_OK;
 }
+int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
+                   float* scores, int32_t* kept_idx, void* stream) {
+  return rs_select_topk_ex(partials, num_partials, B, L, keep_k, RS_DIST_L2, 0, scores, kept_idx,
+                           stream);
+}
 
-int rs_select_gather(const float* partials, int num_partials, const void* y, int B, int L, int C,
-                     int keep_k, float* scores, int32_t* kept_idx, void* y_kept, void* stream) {
+int rs_select_gather_ex(const float* partials, int num_partials, const void* y, int B, int L,
+                        int C, int keep_k, int distance, int flags, float* scores,
+                        int32_t* kept_idx, void* y_kept, void* stream) {
+  RS_TRY(check_mode(distance, flags));
   RS_TRY(check_width(C));
-  if (B < 0 || L < 1 || L > RS_MAX_L || num_partials < 1 || num_partials > 64)
-    return RS_ERR_SHAPE;
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_partials(num_partials, distance));
   RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, num_partials));
-  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  RS_TRY(check_keep(keep_k, L, flags));
   if (B == 0) return RS_OK;
-  if (!partials || !y || !scores || !kept_idx || !y_kept) return RS_ERR_NULL;
+  if (!partials || !y || !scores ||
+      (keep_k + !(flags & RS_NO_CLS) > 0 && (!kept_idx || !y_kept)))
+    return RS_ERR_NULL;
   if (!al4(partials) || !al16(y) || !al4(scores) || !al4(kept_idx) || !al16(y_kept))
     return RS_ERR_ALIGN;
   int num_sms = 148;
@@ -461,9 +503,15 @@ int rs_select_gather(const float* partials, int num_partials, const void* y, int
     RS_TRY(dev_state(&st));
     num_sms = st->num_sms;
   }
-  RS_CUDA(rs::launch_select_gather(partials, num_partials, y, B, L, C, keep_k, scores, kept_idx,
-                                   y_kept, num_sms, static_cast<cudaStream_t>(stream)));
+  RS_CUDA(rs::launch_select_gather(partials, num_partials, y, B, L, C, keep_k, distance,
+                                   !(flags & RS_NO_CLS), scores, kept_idx, y_kept, num_sms,
+                                   static_cast<cudaStream_t>(stream)));
   return RS_OK;
+}
+int rs_select_gather(const float* partials, int num_partials, const void* y, int B, int L, int C,
+                     int keep_k, float* scores, int32_t* kept_idx, void* y_kept, void* stream) {
+  return rs_select_gather_ex(partials, num_partials, y, B, L, C, keep_k, RS_DIST_L2, 0, scores,
+                             kept_idx, y_kept, stream);
 }
 
 int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
@@ -482,22 +530,26 @@ int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, 
     RS_TRY(dev_state(&st));
     num_sms = st->num_sms;
   }
-  RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k, y_kept, num_sms,
+  RS_CUDA(rs::launch_gather(y, B, L, C, kept_idx, keep_k + 1, y_kept, num_sms,
                             static_cast<cudaStream_t>(stream)));
   return RS_OK;
 }
 
-int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, const void* b1,
-                     const void* W2, const void* b2, const void* gamma, const void* beta,
-                     int keep_k, void* y_kept, int32_t* kept_idx, float* scores, void* stream) {
+int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W1,
+                        const void* b1, const void* W2, const void* b2, const void* gamma,
+                        const void* beta, int keep_k, int distance, int flags, void* y_kept,
+                        int32_t* kept_idx, float* scores, void* stream) {
+  RS_TRY(check_mode(distance, flags));
   if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
   RS_TRY(check_width(C));
   RS_TRY(check_hidden(H));
   const int64_t M64 = static_cast<int64_t>(B) * L;
   RS_TRY(check_rows(M64, C, H));
-  if (keep_k < 0 || keep_k > L - 1) return RS_ERR_KEEP_K;
+  RS_TRY(check_keep(keep_k, L, flags));
   if (B == 0) return RS_OK;
-  if (!x || !W1 || !b1 || !W2 || !b2 || !gamma || !beta || !y_kept || !kept_idx || !scores)
+  const bool rows_out = keep_k + !(flags & RS_NO_CLS) > 0;  // any kept row per sample
+  if (!x || !W1 || !b1 || !W2 || !b2 || !gamma || !beta || !scores ||
+      (rows_out && (!y_kept || !kept_idx)))
     return RS_ERR_NULL;
   if (!al16(x) || !al16(W1) || !al16(b1) || !al16(W2) || !al16(b2) || !al16(gamma) ||
       !al16(beta) || !al16(y_kept) || !al4(kept_idx) || !al4(scores))
@@ -514,13 +566,21 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
   void* hidden = ws + w.hidden;
   void* y = ws + w.y;
   float* partials = reinterpret_cast<float*>(ws + w.partials);
-  const int np = rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
+  const int np =
+      rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
 
   RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
-  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, s, /*pdl=*/true));
-  RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, scores, kept_idx, y_kept,
-                                   st->num_sms, s, /*pdl=*/true));
+  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, distance, s, /*pdl=*/true));
+  RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, distance,
+                                   !(flags & RS_NO_CLS), scores, kept_idx, y_kept, st->num_sms, s,
+                                   /*pdl=*/true));
   return RS_OK;
+}
+int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, const void* b1,
+                     const void* W2, const void* b2, const void* gamma, const void* beta,
+                     int keep_k, void* y_kept, int32_t* kept_idx, float* scores, void* stream) {
+  return rs_block_forward_ex(x, B, L, C, H, W1, b1, W2, b2, gamma, beta, keep_k, RS_DIST_L2, 0,
+                             y_kept, kept_idx, scores, stream);
 }
 
 int rs_get_last_device_error(void* stream) {

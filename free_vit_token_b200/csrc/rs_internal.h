@@ -25,6 +25,13 @@ constexpr int kEpiBoxCols = 16;
 // fc2 writes this many shift partials per row and 128 x BN output tile (one per
 // epilogue column group).
 constexpr int kFc2PartialsPerTile = 2;
+// Shift distances (§3.3 "Distance metrics"): the values of rs.h's RS_DIST_*. fc2
+// writes one partial per column group for L2 (sum of squares) and L1 (sum of
+// absolute values), three for cosine (sum h.x, sum h.h, sum x.x).
+constexpr int kDistL2 = 0;
+constexpr int kDistL1 = 1;
+constexpr int kDistCos = 2;
+inline int dist_partials(int dist) { return dist == kDistCos ? 3 : 1; }
 
 // Launches `kern` on `stream`; with `pdl` the launch may begin while the
 // previous kernel in the stream is still running (every kernel of this library
@@ -79,6 +86,7 @@ struct MlpParams {
   unsigned long long timeout_ns;  // limit of one pipeline wait
   int debug_skip_kb;              // test hook: CTA 0 skips this k-block's loads of its
                                   // first tile (-1: off)
+  int dist;                       // fc2: kDistL2, kDistL1 or kDistCos
 };
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);
@@ -117,13 +125,19 @@ cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream);
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
                        const MlpParams& p, int bn, bool pair, int num_sms, cudaStream_t s,
                        bool pdl = false);
+// Selection: `dist` says how partials make a score (kDist*), `cls` whether t = 0 is a
+// CLS token (kept first, never ranked) or ranked like the others. kept_idx holds
+// cls + keep_k entries per sample.
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
-                          float* scores, int32_t* kept_idx, cudaStream_t stream, bool pdl = false);
-cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
+                          int dist, bool cls, float* scores, int32_t* kept_idx,
+                          cudaStream_t stream, bool pdl = false);
+// Gathers k1 rows per sample (k1 = entries of kept_idx per sample).
+cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int k1,
                           void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);
 // Selection then gather in one kernel (B x S CTAs; every CTA of a sample selects).
 cudaError_t launch_select_gather(const float* partials, int num_partials, const void* y, int B,
-                                 int L, int C, int keep_k, float* scores, int32_t* kept_idx,
-                                 void* y_kept, int num_sms, cudaStream_t stream, bool pdl = false);
+                                 int L, int C, int keep_k, int dist, bool cls, float* scores,
+                                 int32_t* kept_idx, void* y_kept, int num_sms,
+                                 cudaStream_t stream, bool pdl = false);
 
 }  // namespace rs

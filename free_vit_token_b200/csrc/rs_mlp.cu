@@ -8,7 +8,9 @@
 //   fc1 (staged LN):           a = GELU(LN(x') W1^T + b1); A = x' tiles (TMA)
 //        normalised in place in shared memory by LN warps before the MMA.
 //   fc2:  h = a W2^T + b2; y = x' + h;          A = a tiles (TMA)
-//         P[r, j] = sum_{c in group j} (h - x')^2   -- Eq. (4) with D = L2
+//         P[r, j] = sum_{c in group j} (h - x')^2   -- Eq. (4) with D = L2, or with
+//         the L1 and cosine distances of §3.3: sum |h - x'|, or the triple
+//         (sum h x', sum h^2, sum x'^2) per column group
 //
 // One CTA per SM loops over 128 x BN output tiles. Warp roles:
 //   warp 0      TMA producer (A and B tiles, 64-wide K blocks, STAGES deep ring)
@@ -443,7 +445,8 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
                              static_cast<uint32_t>(acc * BN + grp * kCols);
       const int col0 = n_blk * BN + grp * kCols;
       const uint32_t vec_u32 = smem_u32(sVec + acc * kVecStride);
-      float part = 0.f;
+      float part = 0.f;                      // L2: sum (h - x')^2; L1: sum |h - x'|
+      float c_hx = 0.f, c_hh = 0.f, c_xx = 0.f;  // cosine: sum h x', sum h^2, sum x'^2
       uint64_t nmu2 = 0, rs2 = 0;  // folded LN: (-mean, -mean), (rstd, rstd) of this row
       if constexpr (EPI == kEpiGeluFold) {
         float2 st = make_float2(0.f, 0.f);
@@ -540,15 +543,42 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
             }
           } else {
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
+            // h in fp32 before rounding; the distance is uniform over the launch
+            if (p.dist == kDistCos) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
-              const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-              const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-              outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
-              const float d0 = h0 - x0, d1 = h1 - x1;
-              part = fmaf(d0, d0, part);
-              part = fmaf(d1, d1, part);
+              for (int e = 0; e < 8; ++e) {
+                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
+                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
+                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
+                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
+                c_hx = fmaf(h0, x0, c_hx);
+                c_hx = fmaf(h1, x1, c_hx);
+                c_hh = fmaf(h0, h0, c_hh);
+                c_hh = fmaf(h1, h1, c_hh);
+                c_xx = fmaf(x0, x0, c_xx);
+                c_xx = fmaf(x1, x1, c_xx);
+              }
+            } else if (p.dist == kDistL1) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
+                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
+                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
+                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
+                part += fabsf(h0 - x0);
+                part += fabsf(h1 - x1);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
+                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
+                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
+                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
+                const float d0 = h0 - x0, d1 = h1 - x1;
+                part = fmaf(d0, d0, part);
+                part = fmaf(d1, d1, part);
+              }
             }
           }
         }
@@ -572,8 +602,17 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         }
       }
       if constexpr (EPI == kEpiResidShift) {
-        if (row_ok)
-          p.partials[static_cast<size_t>(row) * p.num_partials + n_blk * kGroups + grp] = part;
+        if (row_ok) {
+          float* pr = p.partials + static_cast<size_t>(row) * p.num_partials;
+          const int g = n_blk * kGroups + grp;  // column group of the row
+          if (p.dist == kDistCos) {
+            pr[3 * g] = c_hx;
+            pr[3 * g + 1] = c_hh;
+            pr[3 * g + 2] = c_xx;
+          } else {
+            pr[g] = part;
+          }
+        }
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }

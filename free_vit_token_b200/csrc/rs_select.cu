@@ -3,11 +3,14 @@
 // Compression with FlashAttention", §3.1 pruned set x-tilde, §3.2 Eq. (4) and
 // "dropped the tokens having the lowest k scores").
 //
-// Scores: s_t = sqrt(sum_j P[t, j]) in fp32, partials added left to right.
+// Scores in fp32, partials added left to right (§3.3 "Distance metrics"):
+// L2 s_t = sqrt(sum_j P[t, j]); L1 s_t = sum_j P[t, j]; cosine, from per-group
+// triples (h.x, h.h, x.x): s_t = max(0, 1 - HX / max(sqrt(HH) sqrt(XX), 1e-8)).
 // Selection compares fp32 score bits (non-negative floats order like their bit
 // patterns). Token u beats token t when key_u > key_t, or key_u == key_t and
-// u < t; the kept set is the k patch tokens (t = 1..L-1) beaten by fewer than k
-// others, written as [0] ++ ascending(kept t) -- CLS first, never ranked.
+// u < t; the kept set is the k ranked tokens beaten by fewer than k others. With a
+// CLS token the ranked tokens are t = 1..L-1 and the list is [0] ++ ascending(kept
+// t) -- CLS first, never ranked; without, all L tokens are ranked.
 //   * L <= 256: every thread holds one key and counts its beaters in one sweep
 //     over shared memory; an ordered ballot compaction follows.
 //   * longer L: a 4-pass MSB-first radix select finds the k-th largest key T
@@ -84,13 +87,13 @@ __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t* s_
   return res;
 }
 
-// Number of patch tokens u in 1..L-1 that beat key `key` of token t (t >= 1):
-// key_u >= key for u < t, key_u > key for u > t (u = t never counts). The sweep
-// is split at t so every key costs one compare. s_key holds L keys padded with
-// zeros to a multiple of 4: a zero pad lies above t and is never > key. The CLS
-// slot (u = 0 < t) counted exactly when key_0 >= key and is removed.
+// Number of ranked tokens u that beat key `key` of token t: key_u >= key for
+// u < t, key_u > key for u > t (u = t never counts). The sweep is split at t so
+// every key costs one compare. s_key holds L keys padded with zeros to a multiple
+// of 4: a zero pad lies above t and is never > key. With a CLS token (cls), the
+// CLS slot (u = 0 < t, counted exactly when key_0 >= key) is removed.
 __device__ __forceinline__ uint32_t count_beaters(const uint32_t* s_key, int L, uint32_t key,
-                                                  int t) {
+                                                  int t, bool cls) {
   const uint4* k4 = reinterpret_cast<const uint4*>(s_key);
   const int q = (L + 3) >> 2;
   const int qt = t >> 2;  // the quad holding t
@@ -113,7 +116,7 @@ __device__ __forceinline__ uint32_t count_beaters(const uint32_t* s_key, int L, 
     const uint4 v = k4[i];
     n += (v.x > key) + (v.y > key) + (v.z > key) + (v.w > key);
   }
-  return n - (s_key[0] >= key);  // CLS is never ranked
+  return cls ? n - (s_key[0] >= key) : n;  // CLS is never ranked
 }
 
 // Shared memory of one selecting CTA.
@@ -142,22 +145,41 @@ __device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, 
 // Each thread takes rows t = base + tid + i * nt (i < 4) per round and issues all
 // of their loads before adding; the fp32 additions of a row run left to right.
 __device__ __forceinline__ void load_keys(const float* __restrict__ partials, int NP, int L, int b,
-                                          float* __restrict__ scores, const SelSmem& s) {
+                                          float* __restrict__ scores, const SelSmem& s, int dist,
+                                          int first) {
   const int Lpad = (L + 3) & ~3;
   const int tid = threadIdx.x, nt = blockDim.x;
   const float* P = partials + static_cast<size_t>(b) * L * NP;
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // over this thread's patch keys (t >= 1)
-  auto finish = [&](int t, float acc) {
-    const float v = sqrtf(acc);
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // over this thread's ranked keys (t >= first)
+  auto store = [&](int t, float v) {
     if (scores != nullptr) scores[static_cast<size_t>(b) * L + t] = v;
     const uint32_t key = __float_as_uint(v);
     s.key[t] = key;
-    if (t >= 1) {
+    if (t >= first) {
       kmin = key < kmin ? key : kmin;
       kmax = key > kmax ? key : kmax;
     }
   };
-  if ((NP & 3) == 0 && NP <= 8) {
+  // L2: sqrt of the summed squares; L1: the sum itself
+  auto finish = [&](int t, float acc) { store(t, dist == kDistL2 ? sqrtf(acc) : acc); };
+  if (dist == kDistCos) {
+    // per-group triples (h.x, h.h, x.x), each component summed left to right
+    for (int t = tid; t < Lpad; t += nt) {
+      if (t < L) {
+        const float* pr = P + static_cast<size_t>(t) * NP;
+        float hx = 0.f, hh = 0.f, xx = 0.f;
+        for (int j = 0; j < NP; j += 3) {
+          hx += __ldg(pr + j);
+          hh += __ldg(pr + j + 1);
+          xx += __ldg(pr + j + 2);
+        }
+        const float den = fmaxf(sqrtf(hh) * sqrtf(xx), 1e-8f);
+        store(t, fmaxf(1.0f - hx / den, 0.f));
+      } else {
+        s.key[t] = 0u;
+      }
+    }
+  } else if ((NP & 3) == 0 && NP <= 8) {
     // NP a multiple of 4: every row 16-byte aligned, one or two quad loads per row
     const int np4 = NP >> 2;
     const float4* P4 = reinterpret_cast<const float4*>(P);
@@ -246,10 +268,11 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
 
 // The kept list of one sample into s.kept. Every thread of the block calls it;
 // it ends with a barrier, so s.kept is complete on return.
-__device__ void select_into_smem(int L, int k, const SelSmem& s) {
+__device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) s.kept[0] = 0;
+  const int first = cls ? 1 : 0;  // first ranked token; also the kept list's offset
+  if (tid == 0 && cls) s.kept[0] = 0;
   if (k == 0) {
     __syncthreads();
     return;
@@ -258,19 +281,19 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
     const int t = tid;
     const uint32_t key = t < L ? s.key[t] : 0u;
     const bool keep =
-        t >= 1 && t < L && count_beaters(s.key, L, key, t) < static_cast<uint32_t>(k);
+        t >= first && t < L && count_beaters(s.key, L, key, t, cls) < static_cast<uint32_t>(k);
     uint32_t total;
     const uint32_t pos = block_exclusive_count(keep, s.warp, total);
-    if (keep) s.kept[1 + pos] = t;
+    if (keep) s.kept[first + pos] = t;
     __syncthreads();
     return;
   }
-  // Radix select of the k-th largest key among t = 1..L-1. Each round of a pass
+  // Radix select of the k-th largest key among t = first..L-1. Each round of a pass
   // gives thread tid the four keys t = base + 4 tid .. +3 (one 16-byte load).
   const int Lpad = (L + 3) & ~3;
   const uint4* key4 = reinterpret_cast<const uint4*>(s.key);
   uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
-  // Every patch key lies in [kmin, kmax] (as unsigned integers), so the leading bits
+  // Every ranked key lies in [kmin, kmax] (as unsigned integers), so the leading bits
   // on which kmin and kmax agree are those of every key: such digits are taken
   // without a histogram pass (typically the top byte: sign and high exponent bits).
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -296,7 +319,7 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = t0 + i;
-          const bool cand = t >= 1 && t < L;
+          const bool cand = t >= first && t < L;
           const uint32_t digit = cand ? (u[i] >> 24) : 256u;
           const uint32_t peers = __match_any_sync(0xffffffffu, digit);
           if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
@@ -306,7 +329,8 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = t0 + i;
-          if (t >= 1 && t < L && (u[i] & mask) == prefix) atomicAdd(&s.hist[(u[i] >> shift) & 0xFFu], 1u);
+          if (t >= first && t < L && (u[i] & mask) == prefix)
+            atomicAdd(&s.hist[(u[i] >> shift) & 0xFFu], 1u);
         }
       }
     }
@@ -344,7 +368,7 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
     mask |= 0xFFu << shift;
     need -= s.sel[1];
   }
-  // Ordered compaction: token t (1 <= t < L) is kept when key_t > T, or key_t == T
+  // Ordered compaction: token t (first <= t < L) is kept when key_t > T, or key_t == T
   // and fewer than `need` equal keys precede it; its place among the kept tokens
   // is (#keys > T before t) + min(#keys == T before t, need). One packed scan per
   // round counts both (> T in the low half, == T in the high half).
@@ -358,7 +382,7 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = t0 + i;
-      if (t >= 1 && t < L) {
+      if (t >= first && t < L) {
         gt_m |= static_cast<uint32_t>(u[i] > T) << i;
         eq_m |= static_cast<uint32_t>(u[i] == T) << i;
       }
@@ -371,7 +395,7 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t gt = (gt_m >> i) & 1u, eq = (eq_m >> i) & 1u;
-      if (gt || (eq && eqb < need)) s.kept[1 + gtb + (eqb < need ? eqb : need)] = t0 + i;
+      if (gt || (eq && eqb < need)) s.kept[first + gtb + (eqb < need ? eqb : need)] = t0 + i;
       gtb += gt;
       eqb += eq;
     }
@@ -382,7 +406,8 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s) {
 }
 
 __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ partials, int NP,
-                                                      int L, int k, float* __restrict__ scores,
+                                                      int L, int k, int dist, bool cls,
+                                                      float* __restrict__ scores,
                                                       int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
@@ -390,10 +415,11 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
   pdl_wait();
   const int b = blockIdx.x;
   const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
-  load_keys(partials, NP, L, b, scores, s);
-  select_into_smem(L, k, s);
-  int32_t* out = kept + static_cast<size_t>(b) * (k + 1);
-  for (int i = threadIdx.x; i <= k; i += blockDim.x) out[i] = s.kept[i];
+  load_keys(partials, NP, L, b, scores, s, dist, cls ? 1 : 0);
+  select_into_smem(L, k, s, cls);
+  const int k1 = k + (cls ? 1 : 0);
+  int32_t* out = kept + static_cast<size_t>(b) * k1;
+  for (int i = threadIdx.x; i < k1; i += blockDim.x) out[i] = s.kept[i];
 }
 
 // Copies kept rows r = r_first, r_first + r_step, ... (r < k1) of sample b; a warp
@@ -445,8 +471,9 @@ constexpr int kSelGatherThreads = 512;
 // row data per lane need more than half of an SM's register file.
 template <int VPL>
 __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_gather_kernel(
-    const float* __restrict__ partials, int NP, int L, int k, const uint4* __restrict__ y, int Cv,
-    int S, float* __restrict__ scores, int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
+    const float* __restrict__ partials, int NP, int L, int k, int dist, bool cls,
+    const uint4* __restrict__ y, int Cv, int S, float* __restrict__ scores,
+    int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
   pdl_trigger();
@@ -454,9 +481,9 @@ __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_ga
   const int b = blockIdx.x / S, j0 = blockIdx.x % S;
   const bool writer = j0 == 0;
   const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
-  load_keys(partials, NP, L, b, writer ? scores : nullptr, s);
-  select_into_smem(L, k, s);
-  const int k1 = k + 1;
+  load_keys(partials, NP, L, b, writer ? scores : nullptr, s, dist, cls ? 1 : 0);
+  select_into_smem(L, k, s, cls);
+  const int k1 = k + (cls ? 1 : 0);
   if (writer)
     for (int i = threadIdx.x; i < k1; i += blockDim.x)
       kept[static_cast<size_t>(b) * k1 + i] = s.kept[i];
@@ -480,20 +507,22 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ y
     copy_rows<VPL>(y, L, Cv, b, k1, kept, false, gw % per_sample, per_sample, out);
 }
 
+// Keys (L, padded) and the kept list (at most k + 1 entries).
 static size_t select_smem(int L, int k) {
   return static_cast<size_t>((L + 3) & ~3) * 4 + static_cast<size_t>(k + 1) * 4;
 }
 
 cudaError_t launch_select(const float* partials, int num_partials, int B, int L, int keep_k,
-                          float* scores, int32_t* kept_idx, cudaStream_t stream, bool pdl) {
+                          int dist, bool cls, float* scores, int32_t* kept_idx,
+                          cudaStream_t stream, bool pdl) {
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L - 1)));
+                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L)));
   if (e != cudaSuccess) return e;
   int threads = ((L + 31) / 32) * 32;
   if (threads < 64) threads = 64;
   if (L > kRankMaxL) threads = 1024;
   return launch(select_kernel, B, threads, select_smem(L, keep_k), stream, pdl, partials,
-                num_partials, L, keep_k, scores, kept_idx);
+                num_partials, L, keep_k, dist, cls, scores, kept_idx);
 }
 
 template <int VPL>
@@ -503,10 +532,10 @@ static cudaError_t launch_gather_t(const void* y, int B, int L, int Cv, const in
                 Cv, kept_idx, k1, B, static_cast<uint4*>(y_kept));
 }
 
-cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int keep_k,
+cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kept_idx, int k1,
                           void* y_kept, int num_sms, cudaStream_t stream, bool pdl) {
   const int Cv = C / 8;
-  const int k1 = keep_k + 1;
+  if (k1 <= 0) return cudaSuccess;
   int blocks = (B * k1 + 7) / 8;
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   const int vpl = (Cv + 31) / 32;
@@ -517,38 +546,40 @@ cudaError_t launch_gather(const void* y, int B, int L, int C, const int32_t* kep
 }
 
 template <int VPL>
-static cudaError_t launch_sg_t(const float* partials, int NP, int L, int k, const void* y, int Cv,
-                               int B, int S, float* scores, int32_t* kept, void* y_kept,
-                               cudaStream_t stream, bool pdl) {
+static cudaError_t launch_sg_t(const float* partials, int NP, int L, int k, int dist, bool cls,
+                               const void* y, int Cv, int B, int S, float* scores, int32_t* kept,
+                               void* y_kept, cudaStream_t stream, bool pdl) {
   auto kern = select_gather_kernel<VPL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L - 1)));
+                                       static_cast<int>(select_smem(RS_MAX_L, RS_MAX_L)));
   if (e != cudaSuccess) return e;
   return launch(kern, B * S, kSelGatherThreads, select_smem(L, k), stream, pdl, partials, NP, L, k,
-                static_cast<const uint4*>(y), Cv, S, scores, kept, static_cast<uint4*>(y_kept));
+                dist, cls, static_cast<const uint4*>(y), Cv, S, scores, kept,
+                static_cast<uint4*>(y_kept));
 }
 
 cudaError_t launch_select_gather(const float* partials, int num_partials, const void* y, int B,
-                                 int L, int C, int keep_k, float* scores, int32_t* kept_idx,
-                                 void* y_kept, int num_sms, cudaStream_t stream, bool pdl) {
+                                 int L, int C, int keep_k, int dist, bool cls, float* scores,
+                                 int32_t* kept_idx, void* y_kept, int num_sms,
+                                 cudaStream_t stream, bool pdl) {
   // CTAs per sample: about one CTA per SM when B is small, one per sample otherwise
-  const int k1 = keep_k + 1;
+  const int k1 = keep_k + (cls ? 1 : 0);
   int S = num_sms / B;
   if (S > k1) S = k1;
   if (S < 1) S = 1;
   const int Cv = C / 8;
   const int vpl = (Cv + 31) / 32;
   if (vpl <= 1)
-    return launch_sg_t<1>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
-                          stream, pdl);
+    return launch_sg_t<1>(partials, num_partials, L, keep_k, dist, cls, y, Cv, B, S, scores,
+                          kept_idx, y_kept, stream, pdl);
   if (vpl <= 2)
-    return launch_sg_t<2>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
-                          stream, pdl);
+    return launch_sg_t<2>(partials, num_partials, L, keep_k, dist, cls, y, Cv, B, S, scores,
+                          kept_idx, y_kept, stream, pdl);
   if (vpl <= 4)
-    return launch_sg_t<4>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
-                          stream, pdl);
-  return launch_sg_t<8>(partials, num_partials, L, keep_k, y, Cv, B, S, scores, kept_idx, y_kept,
-                        stream, pdl);
+    return launch_sg_t<4>(partials, num_partials, L, keep_k, dist, cls, y, Cv, B, S, scores,
+                          kept_idx, y_kept, stream, pdl);
+  return launch_sg_t<8>(partials, num_partials, L, keep_k, dist, cls, y, Cv, B, S, scores,
+                        kept_idx, y_kept, stream, pdl);
 }
 
 }  // namespace rs

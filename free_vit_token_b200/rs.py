@@ -37,6 +37,12 @@ SIGNATURES = {
     "rs_fc1_gelu_folded": (_i, [_vp, _fp, _vp, _fp, _fp, _i, _i, _i, _vp, _vp]),
     "rs_ln_fc1_gelu_noalloc": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_fc2_residual_shift": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
+    "rs_fc2_residual_shift_ex": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _fp, _vp]),
+    "rs_num_partials_ex": (_i, [_i, _i]),
+    "rs_block_forward_ex": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
+                                 _vp, _ip, _fp, _vp]),
+    "rs_select_topk_ex": (_i, [_fp, _i, _i, _i, _i, _i, _i, _fp, _ip, _vp]),
+    "rs_select_gather_ex": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
     "rs_num_partials": (_i, [_i]),
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
@@ -97,23 +103,36 @@ def _stream(stream) -> Optional[int]:
     return int(stream) or None
 
 
+RS_DIST_L2, RS_DIST_L1, RS_DIST_COSINE = 0, 1, 2
+RS_NO_CLS = 1
+DISTANCES = {"l2": RS_DIST_L2, "l1": RS_DIST_L1, "cosine": RS_DIST_COSINE}
+
+
+def _dist(distance) -> int:
+    return DISTANCES[distance] if isinstance(distance, str) else int(distance)
+
+
 def rs_block_forward(x: torch.Tensor, W1, b1, W2, b2, gamma, beta, keep_k: int,
                      y_kept: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
-                     scores: Optional[torch.Tensor] = None, stream=None
-                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """x [B, L, C] bf16 -> (y_kept [B, 1+k, C] bf16, kept_idx [B, 1+k] int32, scores [B, L] fp32)."""
+                     scores: Optional[torch.Tensor] = None, stream=None, distance="l2",
+                     cls: bool = True) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """x [B, L, C] bf16 -> (y_kept [B, n, C] bf16, kept_idx [B, n] int32, scores [B, L] fp32)
+    with n = 1 + k (CLS first) or k (cls=False: all L tokens ranked). `distance`: "l2",
+    "l1" or "cosine" (or an RS_DIST_* value)."""
     B, L, C = x.shape
     H = W1.shape[0]
     dev = x.device
+    n = keep_k + (1 if cls else 0)
     if y_kept is None:
-        y_kept = torch.empty(B, keep_k + 1, C, dtype=torch.bfloat16, device=dev)
+        y_kept = torch.empty(B, n, C, dtype=torch.bfloat16, device=dev)
     if kept_idx is None:
-        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
+        kept_idx = torch.empty(B, n, dtype=torch.int32, device=dev)
     if scores is None:
         scores = torch.empty(B, L, dtype=torch.float32, device=dev)
-    st = lib().rs_block_forward(_ptr(x), B, L, C, H, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
-                                _ptr(gamma), _ptr(beta), int(keep_k), _ptr(y_kept),
-                                _ptr(kept_idx), _ptr(scores), _stream(stream))
+    st = lib().rs_block_forward_ex(_ptr(x), B, L, C, H, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                                   _ptr(gamma), _ptr(beta), int(keep_k), _dist(distance),
+                                   0 if cls else RS_NO_CLS, _ptr(y_kept), _ptr(kept_idx),
+                                   _ptr(scores), _stream(stream))
     _check(st, "rs_block_forward")
     return y_kept, kept_idx, scores
 
@@ -209,56 +228,60 @@ def rs_gelu_apply(z: torch.Tensor, out: Optional[torch.Tensor] = None, stream=No
     return out
 
 
-def rs_num_partials(C: int) -> int:
-    return int(lib().rs_num_partials(int(C)))
+def rs_num_partials(C: int, distance="l2") -> int:
+    return int(lib().rs_num_partials_ex(int(C), _dist(distance)))
 
 
 def rs_fc2_residual_shift(hidden: torch.Tensor, x2d: torch.Tensor, W2, b2,
                           y: Optional[torch.Tensor] = None, partials: Optional[torch.Tensor] = None,
-                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                          stream=None, distance="l2") -> Tuple[torch.Tensor, torch.Tensor]:
     M, H = hidden.shape
     C = x2d.shape[1]
     if y is None:
         y = torch.empty(M, C, dtype=torch.bfloat16, device=x2d.device)
     if partials is None:
-        partials = torch.empty(M, rs_num_partials(C), dtype=torch.float32, device=x2d.device)
-    st = lib().rs_fc2_residual_shift(_ptr(hidden), _ptr(x2d), M, C, H, _ptr(W2), _ptr(b2), _ptr(y),
-                                     _ptr(partials), _stream(stream))
+        partials = torch.empty(M, rs_num_partials(C, distance), dtype=torch.float32,
+                               device=x2d.device)
+    st = lib().rs_fc2_residual_shift_ex(_ptr(hidden), _ptr(x2d), M, C, H, _ptr(W2), _ptr(b2),
+                                        _dist(distance), _ptr(y), _ptr(partials), _stream(stream))
     _check(st, "rs_fc2_residual_shift")
     return y, partials
 
 
 def rs_select_topk(partials: torch.Tensor, B: int, L: int, keep_k: int,
                    scores: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
-                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                   stream=None, distance="l2", cls: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
     P = partials.shape[-1]
     dev = partials.device
     if scores is None:
         scores = torch.empty(B, L, dtype=torch.float32, device=dev)
     if kept_idx is None:
-        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
-    st = lib().rs_select_topk(_ptr(partials), P, B, L, int(keep_k), _ptr(scores), _ptr(kept_idx),
-                              _stream(stream))
+        kept_idx = torch.empty(B, keep_k + (1 if cls else 0), dtype=torch.int32, device=dev)
+    st = lib().rs_select_topk_ex(_ptr(partials), P, B, L, int(keep_k), _dist(distance),
+                                 0 if cls else RS_NO_CLS, _ptr(scores), _ptr(kept_idx),
+                                 _stream(stream))
     _check(st, "rs_select_topk")
     return scores, kept_idx
 
 
 def rs_select_gather(partials: torch.Tensor, y: torch.Tensor, keep_k: int,
                      scores: Optional[torch.Tensor] = None, kept_idx: Optional[torch.Tensor] = None,
-                     y_kept: Optional[torch.Tensor] = None, stream=None
-                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                     y_kept: Optional[torch.Tensor] = None, stream=None, distance="l2",
+                     cls: bool = True) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """partials [B*L, P] fp32, y [B, L, C] bf16 -> (scores, kept_idx, y_kept)."""
     B, L, C = y.shape
     P = partials.shape[-1]
     dev = y.device
+    n = keep_k + (1 if cls else 0)
     if scores is None:
         scores = torch.empty(B, L, dtype=torch.float32, device=dev)
     if kept_idx is None:
-        kept_idx = torch.empty(B, keep_k + 1, dtype=torch.int32, device=dev)
+        kept_idx = torch.empty(B, n, dtype=torch.int32, device=dev)
     if y_kept is None:
-        y_kept = torch.empty(B, keep_k + 1, C, dtype=y.dtype, device=dev)
-    st = lib().rs_select_gather(_ptr(partials), P, _ptr(y), B, L, C, int(keep_k), _ptr(scores),
-                                _ptr(kept_idx), _ptr(y_kept), _stream(stream))
+        y_kept = torch.empty(B, n, C, dtype=y.dtype, device=dev)
+    st = lib().rs_select_gather_ex(_ptr(partials), P, _ptr(y), B, L, C, int(keep_k),
+                                   _dist(distance), 0 if cls else RS_NO_CLS, _ptr(scores),
+                                   _ptr(kept_idx), _ptr(y_kept), _stream(stream))
     _check(st, "rs_select_gather")
     return scores, kept_idx, y_kept
 

@@ -47,10 +47,27 @@ extern "C" {
 #define RS_MAX_C 2048
 #define RS_MAX_H 16384
 
+/* Shift distances D of §3.3 "Distance metrics", for the extended (_ex) entry
+ * points; the others use RS_DIST_L2, the paper's default:
+ *   RS_DIST_L2      s = || h - x' ||_2                               (case (i))
+ *   RS_DIST_L1      s = || h - x' ||_1                               (case (ii))
+ *   RS_DIST_COSINE  s = 1 - h.x' / max(||h|| ||x'||, 1e-8), floored  (case (iii))
+ *                   at 0 in fp32 (the pages give neither floor)
+ * with h = MLP(LN(x')) in fp32, before rounding. */
+#define RS_DIST_L2 0
+#define RS_DIST_L1 1
+#define RS_DIST_COSINE 2
+/* Flags of the extended entry points. RS_NO_CLS: t = 0 is an ordinary token
+ * (a video sequence of patch tokens, as UMT's, §4.1): all L tokens are ranked,
+ * 0 <= keep_k <= L, and kept_idx / y_kept hold keep_k entries per sample
+ * instead of 1 + keep_k with the CLS token first. */
+#define RS_NO_CLS 1
+
 typedef enum rs_status {
   RS_OK = 0,
   RS_ERR_NULL = 1,            /* a required pointer is NULL */
-  RS_ERR_SHAPE = 2,           /* B, L, C or H outside the limits above */
+  RS_ERR_SHAPE = 2,           /* B, L, C or H outside the limits above, or an unknown
+                                 distance / flag */
   RS_ERR_KEEP_K = 3,          /* keep_k outside 0..L-1 */
   RS_ERR_ALIGN = 4,           /* a pointer is not 16-byte (tensors) / 4-byte (int, float) aligned */
   RS_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */
@@ -83,6 +100,16 @@ int rs_block_forward(const void* x, int B, int L, int C, int H,
                      const void* W1, const void* b1, const void* W2, const void* b2,
                      const void* gamma, const void* beta, int keep_k,
                      void* y_kept, int32_t* kept_idx, float* scores, void* stream);
+
+/* rs_block_forward with a choice of shift distance (RS_DIST_*) and flags
+ * (RS_NO_CLS). With RS_NO_CLS, 0 <= keep_k <= L and y_kept [B, keep_k, C],
+ * kept_idx [B, keep_k] (may be NULL when keep_k = 0). rs_block_forward is
+ * rs_block_forward_ex(..., RS_DIST_L2, 0, ...). Unknown distance or flags:
+ * RS_ERR_SHAPE. */
+int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W1,
+                        const void* b1, const void* W2, const void* b2, const void* gamma,
+                        const void* beta, int keep_k, int distance, int flags, void* y_kept,
+                        int32_t* kept_idx, float* scores, void* stream);
 
 /*
  * Step-level entry points. rs_block_forward launches exactly these kernels in
@@ -133,10 +160,18 @@ int rs_gelu_apply(const float* z, float* out, int n, void* stream);
 int rs_fc2_residual_shift(const void* hidden, const void* x, int M, int C, int H,
                           const void* W2, const void* b2, void* y, float* partials,
                           void* stream);
+/* The same with the partials of another distance: RS_DIST_L1 sums |h - x'|,
+ * RS_DIST_COSINE writes per column group the triple (sum h x', sum h^2,
+ * sum x'^2); partials is [M, rs_num_partials_ex(C, distance)] fp32. */
+int rs_fc2_residual_shift_ex(const void* hidden, const void* x, int M, int C, int H,
+                             const void* W2, const void* b2, int distance, void* y,
+                             float* partials, void* stream);
 
 /* Number of per-row partial sums rs_fc2_residual_shift writes for width C
- * (0 if C is unsupported). */
+ * (0 if C is unsupported); rs_num_partials_ex: for a distance (three per column
+ * group for RS_DIST_COSINE, one otherwise; 0 for an unknown distance). */
 int rs_num_partials(int C);
+int rs_num_partials_ex(int C, int distance);
 
 /* Score finalisation and per-sample top-k (§3.2 drop the lowest-k scores):
  *   scores[b, t] = sqrt(sum_{j=0..P-1} partials[b*L+t, j])  (fp32, left to right)
@@ -145,6 +180,12 @@ int rs_num_partials(int C);
  * partials [B*L, P] fp32 with 1 <= P <= 64; scores [B, L]; kept_idx [B, 1+keep_k]. */
 int rs_select_topk(const float* partials, int num_partials, int B, int L, int keep_k,
                    float* scores, int32_t* kept_idx, void* stream);
+/* rs_select_topk for another distance and flags: scores are sum_j P (L1) or
+ * max(0, 1 - HX / max(sqrt(HH) sqrt(XX), 1e-8)) from per-group triples summed
+ * component-wise left to right (cosine; num_partials a multiple of 3); with
+ * RS_NO_CLS all L tokens are ranked and kept_idx is [B, keep_k]. */
+int rs_select_topk_ex(const float* partials, int num_partials, int B, int L, int keep_k,
+                      int distance, int flags, float* scores, int32_t* kept_idx, void* stream);
 
 /* rs_select_topk followed by rs_gather_rows (same outputs), as rs_block_forward
  * runs them: for L <= 256 one fused kernel in which every CTA ranks its
@@ -152,6 +193,11 @@ int rs_select_topk(const float* partials, int num_partials, int B, int L, int ke
  * (1 <= P <= 64), y [B, L, C] bf16; outputs as for the two calls. */
 int rs_select_gather(const float* partials, int num_partials, const void* y, int B, int L, int C,
                      int keep_k, float* scores, int32_t* kept_idx, void* y_kept, void* stream);
+/* rs_select_gather for another distance and flags (as rs_select_topk_ex);
+ * y_kept is [B, keep_k + (flags & RS_NO_CLS ? 0 : 1), C]. */
+int rs_select_gather_ex(const float* partials, int num_partials, const void* y, int B, int L,
+                        int C, int keep_k, int distance, int flags, float* scores,
+                        int32_t* kept_idx, void* y_kept, void* stream);
 
 /* Row gather, the pruned set x-tilde (§3.1):
  * y_kept[b, j, :] = y[b, kept_idx[b, j], :]. y [B, L, C] bf16; kept_idx

@@ -31,9 +31,10 @@ def weights64(w):
                 gamma=f64(w.gamma), beta=f64(w.beta))
 
 
-def oracle_block(x_bf16: torch.Tensor, w, keep_k: int):
+def oracle_block(x_bf16: torch.Tensor, w, keep_k: int, metric: str = "l2", cls: bool = True):
     """Oracle on bf16 CPU inputs [B, L, C]: (y_kept, kept, scores, y) in float64."""
-    return oracle.block_forward(f64(x_bf16), keep_k=keep_k, **weights64(w))
+    return oracle.block_forward(f64(x_bf16), keep_k=keep_k, metric=metric, cls=cls,
+                                **weights64(w))
 
 
 def check_y(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = "y") -> float:
@@ -53,28 +54,34 @@ def check_scores(s_gpu: np.ndarray, s_ref: np.ndarray) -> float:
     return float(np.max(d / np.maximum(s_ref, 1e-6)))
 
 
-def check_kept(kept_gpu: np.ndarray, s_ref_row: np.ndarray, kept_ref: np.ndarray, k: int) -> bool:
-    """Returns True when the exact rule applied (False: band rule)."""
+def check_kept(kept_gpu: np.ndarray, s_ref_row: np.ndarray, kept_ref: np.ndarray, k: int,
+               cls: bool = True) -> bool:
+    """Returns True when the exact rule applied (False: band rule). With a CLS token
+    the list is [0] ++ k ranked patch tokens; without, k ranked tokens of 0..L-1."""
     L = s_ref_row.shape[0]
+    first = 1 if cls else 0
     kg = [int(v) for v in kept_gpu]
-    assert len(kg) == k + 1 and kg[0] == 0, kg[:4]
+    assert len(kg) == k + first, (len(kg), k)
+    if cls:
+        assert kg[0] == 0, kg[:4]
+    ranked = kg[first:]
     assert all(kg[i] < kg[i + 1] for i in range(len(kg) - 1)), "kept indices not ascending/unique"
-    assert all(1 <= t < L for t in kg[1:])
-    if k == 0 or k == L - 1:
+    assert all(first <= t < L for t in ranked)
+    if k == 0 or k == L - first:
         assert kg == list(kept_ref)
         return True
-    sp = np.sort(s_ref_row[1:])[::-1]
+    sp = np.sort(s_ref_row[first:])[::-1]
     t_k, t_k1 = sp[k - 1], sp[k]
     if (t_k - t_k1) >= GAP_TOL * t_k:
         assert kg == list(kept_ref), "kept_idx differs where the oracle's gap is >= 1e-3"
         return True
-    kept_set = set(kg[1:])
-    dropped = [t for t in range(1, L) if t not in kept_set]
-    assert min(s_ref_row[t] for t in kg[1:]) >= max(s_ref_row[t] for t in dropped) - GAP_TOL * t_k
+    kept_set = set(ranked)
+    dropped = [t for t in range(first, L) if t not in kept_set]
+    assert min(s_ref_row[t] for t in ranked) >= max(s_ref_row[t] for t in dropped) - GAP_TOL * t_k
     return False
 
 
-def check_block(gpu, ref, k: int, samples=None) -> dict:
+def check_block(gpu, ref, k: int, samples=None, cls: bool = True) -> dict:
     """gpu = (y_kept, kept_idx, scores) torch tensors (full batch); ref = oracle output on
     the batch rows listed in ``samples`` (all when None)."""
     y_kept_g, kept_g, s_g = (t.detach().cpu() for t in gpu)
@@ -86,6 +93,8 @@ def check_block(gpu, ref, k: int, samples=None) -> dict:
     worst_s = check_scores(f64(s_g)[samples], s_r)
     for i, b in enumerate(samples):
         kg = kept_g[b].numpy()
-        exact += check_kept(kg, s_r[i], kept_r[i], k)
-        worst_y = max(worst_y, check_y(f64(y_kept_g[b]), y_r[i][kg.astype(np.int64)], f"y_kept[{b}]"))
+        exact += check_kept(kg, s_r[i], kept_r[i], k, cls)
+        if kg.size:  # no kept row at all without CLS and keep_k = 0
+            worst_y = max(worst_y, check_y(f64(y_kept_g[b]), y_r[i][kg.astype(np.int64)],
+                                           f"y_kept[{b}]"))
     return dict(exact=exact, band=len(samples) - exact, worst_y=worst_y, worst_s=worst_s)

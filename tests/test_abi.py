@@ -87,6 +87,34 @@ def test_step_entry_points_argument_errors():
     assert L.rs_gather_rows(FAKE, 2, 10, 192, None, 3, FAKE, None) == rs.RS_ERR_NULL
 
 
+def test_extended_entry_points_argument_errors():
+    L = rs.lib()
+    NO_CLS, COS, L1_ = rs.RS_NO_CLS, rs.RS_DIST_COSINE, rs.RS_DIST_L1
+    assert L.rs_num_partials_ex(384, COS) == 3 * L.rs_num_partials(384) == 12
+    assert L.rs_num_partials_ex(768, L1_) == L.rs_num_partials(768)
+    assert L.rs_num_partials_ex(384, 3) == 0
+    sel = lambda np_, B, Lq, k, d, f, kept=FAKE: L.rs_select_topk_ex(FAKE, np_, B, Lq, k, d, f,
+                                                                      FAKE, kept, None)
+    assert sel(6, 2, 10, 3, 3, 0) == rs.RS_ERR_SHAPE           # unknown distance
+    assert sel(6, 2, 10, 3, 0, 2) == rs.RS_ERR_SHAPE           # unknown flag
+    assert sel(4, 2, 10, 3, COS, 0) == rs.RS_ERR_SHAPE         # cosine partials are triples
+    assert sel(66, 2, 10, 3, COS, 0) == rs.RS_ERR_SHAPE        # more than 64 partials
+    assert sel(6, 2, 10, 10, 0, 0) == rs.RS_ERR_KEEP_K         # keep_k = L needs no CLS
+    assert sel(6, 2, 10, 11, 0, NO_CLS) == rs.RS_ERR_KEEP_K
+    assert sel(6, 0, 10, 10, 0, NO_CLS) == rs.RS_OK            # empty batch
+    assert sel(6, 2, 10, 3, COS, NO_CLS, kept=FAKE + 2) == rs.RS_ERR_ALIGN
+    fwd = lambda k, d, f: L.rs_block_forward_ex(FAKE, 2, 10, 192, 768, FAKE, FAKE, FAKE, FAKE,
+                                                FAKE, FAKE, k, d, f, FAKE, FAKE, FAKE, None)
+    assert fwd(3, 5, 0) == rs.RS_ERR_SHAPE
+    assert fwd(3, 0, 4) == rs.RS_ERR_SHAPE
+    assert fwd(10, 0, 0) == rs.RS_ERR_KEEP_K
+    assert fwd(-1, 0, NO_CLS) == rs.RS_ERR_KEEP_K
+    assert L.rs_fc2_residual_shift_ex(FAKE, FAKE, 10, 192, 768, FAKE, FAKE, 9, FAKE, FAKE,
+                                      None) == rs.RS_ERR_SHAPE
+    assert L.rs_select_gather_ex(FAKE, 6, FAKE, 2, 10, 192, 3, COS, 0, FAKE, FAKE, MIS,
+                                 None) == rs.RS_ERR_ALIGN
+
+
 def test_library_has_no_torch_or_libcuda_link_dependency():
     out = os.popen(f"ldd {rs.LIB_PATH}").read()
     assert "libtorch" not in out and "libc10" not in out
