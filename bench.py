@@ -43,9 +43,9 @@ SG_REPS = 20  # select+gather launches per timing graph
 
 def kernels_per_step(wl) -> int:
     """Kernels rs_block_forward launches per stage: LN prep (statistics + weight
-    fold), fc1, fc2, then one fused select+gather kernel (L <= 256) or select and
-    gather (longer L)."""
-    return sum(4 if wl.stage_L(s) <= 256 else 5 for s in range(wl.stages))
+    fold), fc1, fc2 and the fused select+gather (rank select for L <= 256, radix
+    select above, both inside the same kernel)."""
+    return 4 * wl.stages
 
 
 def load_peaks():
