@@ -48,6 +48,11 @@ def kernels_per_step(wl) -> int:
     return 4 * wl.stages
 
 
+# Datasheet figures, reported beside the measured denominators for context only.
+DATASHEET_BF16_TF = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -473,6 +478,9 @@ def main():
                      "kernel_ms": fc_ms[dominant]},
         "block_tflops": block_flops / (ms_per_step / 1e3) / 1e12,
         "block_frac_of_bf16_peak": block_flops / (ms_per_step / 1e3) / 1e12 / peak_tf,
+        "block_frac_other_peaks": {
+            "bf16_sustained": block_flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_sustained"],
+            "bf16_datasheet_2250": block_flops / (ms_per_step / 1e3) / 1e12 / DATASHEET_BF16_TF},
         "kernel_ms": {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage)
                       for n in names},
         "select_gather": {"GBps": sg_gbs, "frac_hbm": sg_gbs / peaks["hbm"],
@@ -480,6 +488,7 @@ def main():
                           "timing": f"device time per launch, {SG_REPS} launches replayed from a "
                                     "CUDA graph, inputs as fc2 left them (L2-resident)",
                           "ms_single_launch_events": sel_ms_event,
+                          "frac_of_8TBps": sg_gbs / DATASHEET_HBM_GBS,
                           "after_l2_flush": {"ms": sel_ms_flushed,
                                              "GBps": sg_bytes / (sel_ms_flushed / 1e3) / 1e9,
                                              "frac_hbm": sg_bytes / (sel_ms_flushed / 1e3) / 1e9
