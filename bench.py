@@ -197,6 +197,52 @@ def oracle_rate(wl, seed: int, budget_s: float):
 
 
 # ----------------------------------------------------------------------------- main
+def time_attention(rs, wl, x_full, x_kept, peaks, dev, stream, reps: int):
+    """The attention sublayer (x + SA(LN(x)), Eq. (5)) that the next layer runs, on
+    the stage-0 input (L tokens) and on the pruned block's output (1 + k tokens):
+    what the pruning saves downstream. Outside the timed steps; each figure is the
+    mean of `reps` back-to-back calls between CUDA events on the launch stream
+    (inputs L2-warm), and for the attention core alone its FLOP rate against the
+    bf16 peak (4 L^2 C flops per sample: Q K^T and P V)."""
+    if reps <= 0 or wl.C % 64:
+        return None
+    from workloads import draw_attn_weights
+    heads = wl.C // 64
+    w = draw_attn_weights(wl.C, seed=1000)
+    W = [t.to(dev) for t in (w.Wqkv, w.bqkv, w.Wo, w.bo, w.gamma, w.beta)]
+    res = {"heads": heads, "head_dim": 64, "reps": reps,
+           "timing": "mean of back-to-back calls between CUDA events, inputs L2-warm"}
+    for tag, xin in (("full", x_full), ("kept", x_kept)):
+        B, L, C = xin.shape
+        out = torch.empty_like(xin)
+        qkv = torch.randn(B, L, 3 * C, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        core_out = torch.empty(B, L, C, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            rs.rs_attn_sublayer(xin, *W, heads, out=out, stream=stream)
+            rs.rs_attn_core(qkv, heads, out=core_out, stream=stream)
+        torch.cuda.synchronize()
+        t = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        t[0].record(stream)
+        for _ in range(reps):
+            rs.rs_attn_sublayer(xin, *W, heads, out=out, stream=stream)
+        t[1].record(stream)
+        t[2].record(stream)
+        for _ in range(reps):
+            rs.rs_attn_core(qkv, heads, out=core_out, stream=stream)
+        t[3].record(stream)
+        torch.cuda.synchronize()
+        sub_ms = t[0].elapsed_time(t[1]) / reps
+        core_ms = t[2].elapsed_time(t[3]) / reps
+        core_tf = 4.0 * B * L * L * C / (core_ms / 1e3) / 1e12
+        proj_flops = 2.0 * B * L * C * 4 * C
+        res[tag] = {"tokens_per_sample": L, "sublayer_ms": sub_ms, "core_ms": core_ms,
+                    "core_tflops": core_tf, "core_frac_bf16": core_tf / peaks["bf16"],
+                    "sublayer_tflops": (proj_flops + 4.0 * B * L * L * C) / (sub_ms / 1e3) / 1e12}
+    assert rs.rs_get_last_device_error() == 0
+    res["sublayer_speedup_kept_vs_full"] = res["full"]["sublayer_ms"] / res["kept"]["sublayer_ms"]
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -204,6 +250,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="deit_s", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--attn-reps", type=int, default=20,
+                    help="calls per attention-sublayer timing (0: skip that measurement)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline leg (0 = skip)")
     args = ap.parse_args()
@@ -457,6 +505,8 @@ def main():
     e2e_value = job_throughput(tokens_per_step, 1, e2e_ms, world)
     clocks.stop()
 
+    attn = time_attention(rs, wl, x, outs[0][0], peaks, dev, stream, args.attn_reps)
+
     cpu = None
     if rank == 0 and args.cpu_budget > 0:
         r, n, dt, thr = oracle_rate(wl, 0, args.cpu_budget)
@@ -499,6 +549,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (own streams)"},
+        "attention_next_layer": attn,
         "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

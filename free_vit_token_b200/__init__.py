@@ -11,6 +11,9 @@ from .rs import (  # noqa: F401
     RS_NO_CLS,
     RsError,
     lib,
+    rs_attn_core,
+    rs_attn_forward,
+    rs_attn_sublayer,
     rs_block_forward,
     rs_fc2_residual_shift,
     rs_debug_fc1_skip_load,

@@ -164,7 +164,7 @@ int check_rows(int64_t M, int C, int H) {
 // previous work normally; the GEMM is a programmatic dependent launch.
 int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, const void* b1,
             const void* gamma, const void* beta, uint8_t* ws, const WsLayout& w, void* hidden,
-            bool staged, cudaStream_t s) {
+            bool staged, cudaStream_t s, bool linear = false) {
   float* stats = reinterpret_cast<float*>(ws + w.stats);
   const int bn = rs::fc1_block_n(H);
   const bool pair = rs::gemm_pair(M, C, staged);
@@ -179,6 +179,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
+  p.linear = linear ? 1 : 0;
   const void* wB = W1;
   if (staged) {
     RS_CUDA(rs::launch_ln_stats(x, M, C, stats, st.num_sms, s));
@@ -246,6 +247,120 @@ int check_keep(int keep_k, int L, int flags) {
 int check_partials(int num_partials, int distance) {
   if (num_partials < 1 || num_partials > 64) return RS_ERR_SHAPE;
   if (distance == RS_DIST_COSINE && num_partials % 3 != 0) return RS_ERR_SHAPE;
+  return RS_OK;
+}
+
+// ---------------------------------------------------------------- attention sublayer
+// Workspace of the attention sublayer: the QKV projection's LN statistics and
+// folded weights (the fc1 fields of WsLayout), the projection [M, 3C] (`hidden`),
+// x' [M, C] (`y`, pruning variant), the shift partials, and the attention
+// output [M, C] at `o`.
+struct AttnWs {
+  WsLayout w;
+  size_t o;
+};
+AttnWs attn_ws_layout(int64_t M, int C) {
+  AttnWs a{};
+  WsLayout& w = a.w;
+  size_t off = 0;
+  w.stats = off;
+  off = align_up(off + static_cast<size_t>(M) * 8, 1024);
+  w.wg = off;
+  off = align_up(off + static_cast<size_t>(3 * C) * C * 2, 1024);
+  w.colg = off;
+  off = align_up(off + static_cast<size_t>(3 * C) * 4, 1024);
+  w.colc = off;
+  off = align_up(off + static_cast<size_t>(3 * C) * 4, 1024);
+  w.fc1_total = off;
+  w.hidden = off;
+  off = align_up(off + static_cast<size_t>(M) * 3 * C * 2, 1024);
+  w.y = off;
+  off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
+  w.partials = off;
+  off = align_up(off + static_cast<size_t>(M) * rs::dist_partials(rs::kDistCos) *
+                           (rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C)) * 4,
+                 1024);
+  a.o = off;
+  off = align_up(off + static_cast<size_t>(M) * C * 2, 1024);
+  w.total = off;
+  return a;
+}
+
+// The QKV projection [B*L, 3C] as a [B][L][3C] tensor with {64, 128, 1} boxes.
+int make_tmap_qkv(CUtensorMap* m, const void* qkv, int B, int L, int C) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return RS_ERR_CUDA;
+  const cuuint64_t row = static_cast<cuuint64_t>(3 * C) * 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * C), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[2] = {row, row * static_cast<cuuint64_t>(L)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RS_OK : RS_ERR_CUDA;
+}
+
+// Heads of width 64: C = 64 heads, within the library's width limit.
+int check_heads(int C, int heads) {
+  if (heads < 1 || C != 64 * heads) return RS_ERR_SHAPE;
+  return check_width(C);
+}
+
+int run_attn_core(DevState& st, const void* qkv, int B, int L, int C, int heads, void* out,
+                  cudaStream_t s, bool pdl) {
+  CUtensorMap tm;
+  RS_TRY(make_tmap_qkv(&tm, qkv, B, L, C));
+  rs::AttnParams p{};
+  p.B = B;
+  p.L = L;
+  p.C = C;
+  p.heads = heads;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = st.err;
+  p.timeout_ns = rs::kDefaultTimeoutNs;
+  RS_CUDA(rs::launch_attn(tm, p, s, pdl));
+  return RS_OK;
+}
+
+// x_out = x + SA(LN(x)) Wo^T + bo, and the shift partials of D(SA(LN(x)), x):
+// LN prep + QKV projection (the folded-LN GEMM without activation), the
+// attention core, the output projection (the fc2 GEMM with K = C).
+int run_attn_sublayer(DevState& st, const void* x, int B, int L, int C, int heads,
+                      const void* Wqkv, const void* bqkv, const void* Wo, const void* bo,
+                      const void* gamma, const void* beta, void* x_out, int distance,
+                      cudaStream_t s, uint8_t** ws_out, WsLayout* w_out) {
+  const int64_t M64 = static_cast<int64_t>(B) * L;
+  const int M = static_cast<int>(M64);
+  const AttnWs aw = attn_ws_layout(M64, C);
+  const WsLayout& w = aw.w;
+  RS_TRY(ensure_ws(st, w.total));
+  uint8_t* ws = static_cast<uint8_t*>(st.ws);
+  void* qkv = ws + w.hidden;
+  void* attn_o = ws + aw.o;
+  float* partials = reinterpret_cast<float*>(ws + w.partials);
+  RS_TRY(run_fc1(st, x, M, C, 3 * C, Wqkv, bqkv, gamma, beta, ws, w, qkv, false, s,
+                 /*linear=*/true));
+  RS_TRY(run_attn_core(st, qkv, B, L, C, heads, attn_o, s, /*pdl=*/true));
+  RS_TRY(run_fc2(st, attn_o, x, M, C, C, Wo, bo, x_out ? x_out : ws + w.y, partials, distance, s,
+                 /*pdl=*/true));
+  if (ws_out) *ws_out = ws;
+  if (w_out) *w_out = w;
+  return RS_OK;
+}
+
+int check_attn_args(const void* x, int B, int L, int C, int heads, const void* Wqkv,
+                    const void* bqkv, const void* Wo, const void* bo, const void* gamma,
+                    const void* beta) {
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_heads(C, heads));
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, 3 * C));
+  if (B == 0) return RS_OK;
+  if (!x || !Wqkv || !bqkv || !Wo || !bo || !gamma || !beta) return RS_ERR_NULL;
+  if (!al16(x) || !al16(Wqkv) || !al16(bqkv) || !al16(Wo) || !al16(bo) || !al16(gamma) ||
+      !al16(beta))
+    return RS_ERR_ALIGN;
   return RS_OK;
 }
 
@@ -581,6 +696,61 @@ int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, 
                      int keep_k, void* y_kept, int32_t* kept_idx, float* scores, void* stream) {
   return rs_block_forward_ex(x, B, L, C, H, W1, b1, W2, b2, gamma, beta, keep_k, RS_DIST_L2, 0,
                              y_kept, kept_idx, scores, stream);
+}
+
+int rs_attn_core(const void* qkv, int B, int L, int heads, void* out, void* stream) {
+  if (B < 0 || L < 1 || L > RS_MAX_L || heads < 1) return RS_ERR_SHAPE;
+  const int C = 64 * heads;
+  RS_TRY(check_heads(C, heads));
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, 3 * C));
+  if (B == 0) return RS_OK;
+  if (!qkv || !out) return RS_ERR_NULL;
+  if (!al16(qkv) || !al16(out)) return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_attn_core(*st, qkv, B, L, C, heads, out, static_cast<cudaStream_t>(stream), false);
+}
+
+int rs_attn_sublayer(const void* x, int B, int L, int C, int heads, const void* Wqkv,
+                     const void* bqkv, const void* Wo, const void* bo, const void* gamma,
+                     const void* beta, void* x_out, void* stream) {
+  RS_TRY(check_attn_args(x, B, L, C, heads, Wqkv, bqkv, Wo, bo, gamma, beta));
+  if (B == 0) return RS_OK;
+  if (!x_out) return RS_ERR_NULL;
+  if (!al16(x_out)) return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_attn_sublayer(*st, x, B, L, C, heads, Wqkv, bqkv, Wo, bo, gamma, beta, x_out,
+                           RS_DIST_L2, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+int rs_attn_forward_ex(const void* x, int B, int L, int C, int heads, const void* Wqkv,
+                       const void* bqkv, const void* Wo, const void* bo, const void* gamma,
+                       const void* beta, int keep_k, int distance, int flags, void* x_kept,
+                       int32_t* kept_idx, float* scores, void* stream) {
+  RS_TRY(check_mode(distance, flags));
+  RS_TRY(check_attn_args(x, B, L, C, heads, Wqkv, bqkv, Wo, bo, gamma, beta));
+  RS_TRY(check_keep(keep_k, L, flags));
+  if (B == 0) return RS_OK;
+  const bool rows_out = keep_k + !(flags & RS_NO_CLS) > 0;
+  if (!scores || (rows_out && (!x_kept || !kept_idx))) return RS_ERR_NULL;
+  if (!al16(x_kept) || !al4(kept_idx) || !al4(scores)) return RS_ERR_ALIGN;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  uint8_t* ws = nullptr;
+  WsLayout w{};
+  RS_TRY(run_attn_sublayer(*st, x, B, L, C, heads, Wqkv, bqkv, Wo, bo, gamma, beta, nullptr,
+                           distance, s, &ws, &w));
+  const int np =
+      rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
+  RS_CUDA(rs::launch_select_gather(reinterpret_cast<float*>(ws + w.partials), np, ws + w.y, B, L,
+                                   C, keep_k, distance, !(flags & RS_NO_CLS), scores, kept_idx,
+                                   x_kept, st->num_sms, s, /*pdl=*/true));
+  return RS_OK;
 }
 
 int rs_get_last_device_error(void* stream) {

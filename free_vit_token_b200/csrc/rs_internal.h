@@ -87,6 +87,7 @@ struct MlpParams {
   int debug_skip_kb;              // test hook: CTA 0 skips this k-block's loads of its
                                   // first tile (-1: off)
   int dist;                       // fc2: kDistL2, kDistL1 or kDistCos
+  int linear;                     // folded-LN fc1: 0 = erf-GELU, 1 = no activation (QKV)
 };
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);
@@ -139,5 +140,19 @@ cudaError_t launch_select_gather(const float* partials, int num_partials, const 
                                  int L, int C, int keep_k, int dist, bool cls, float* scores,
                                  int32_t* kept_idx, void* y_kept, int num_sms,
                                  cudaStream_t stream, bool pdl = false);
+
+// Attention core (rs_attn.cu): per sample and head of width 64, Softmax(Q K^T / 8) V
+// from a QKV projection [B, L, 3C] (Q, K, V at columns 0, C, 2C; head h at +64 h),
+// written to out [B, L, C] (head h at columns 64 h). The tensor map views the QKV
+// buffer as [B][L][3C] with {64, 128, 1} boxes and the 128-byte swizzle.
+struct AttnParams {
+  int B, L, C, heads;
+  __nv_bfloat16* out;
+  int* err;                       // device status flag
+  unsigned long long timeout_ns;  // limit of one pipeline wait
+};
+size_t attn_smem_bytes();
+cudaError_t launch_attn(const CUtensorMap& tmQKV, const AttnParams& p, cudaStream_t stream,
+                        bool pdl = false);
 
 }  // namespace rs

@@ -513,7 +513,12 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
                 ffma2(nmu2, gb, f2pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]))),
                 cb);
           }
-          gelu2_block<8>(z2, g2);
+          if (!p.linear) {
+            gelu2_block<8>(z2, g2);
+          } else {  // no activation: the attention sublayer's QKV projection
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g2[e] = z2[e];
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float2 g = f2unpack(g2[e]);

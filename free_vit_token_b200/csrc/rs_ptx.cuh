@@ -146,6 +146,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// 3-D tiled load of box {x .. x+box0, y .. y+box1, z .. z+box2}; out-of-range
+// elements read as zero.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 // CTA-pair form: the load lands in this CTA's shared memory and completes its
 // bytes on the mbarrier at `bar_cluster` (a shared::cluster address, here the
 // leader CTA's barrier).
@@ -377,12 +387,39 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major bf16 operand (the N = 64
+// columns of each K row contiguous) in the same TMA 128-byte swizzle layout:
+// K row k at a 128 B pitch, 8-row groups 1024 B apart (stride byte offset), the
+// next 64-element block along N at `mn_stride` bytes (leading byte offset; not
+// read when N = 64). Start on a 1024-byte boundary (+2048 B per 16 K rows).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major,
 // M = 128, N = n (bits: D format 4-5, A format 7-9, B format 10-12, N>>3 at
 // 17-22, M>>4 at 24-28).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// The same with B read MN-major (bit 16, "transpose B").
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int m, int n) {
+  return idesc_bf16_f32(m, n) | (1u << 16);
+}
+
+// 2^x on the SFU (ex2.approx: relative error about 2^-22, 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ---------------------------------------------------------------- paired fp32 (sm_100)

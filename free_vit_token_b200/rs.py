@@ -47,6 +47,10 @@ SIGNATURES = {
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
     "rs_select_gather": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
+    "rs_attn_core": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "rs_attn_sublayer": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "rs_attn_forward_ex": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
+                                _vp, _ip, _fp, _vp]),
     "rs_status_string": (ctypes.c_char_p, [_i]),
     "rs_get_last_device_error": (_i, [_vp]),
     "rs_release_workspace": (None, []),
@@ -307,3 +311,55 @@ def rs_release_workspace() -> None:
 
 def rs_workspace_bytes(B: int, L: int, C: int, H: int) -> int:
     return int(lib().rs_workspace_bytes(B, L, C, H))
+
+
+def rs_attn_core(qkv: torch.Tensor, heads: int, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """qkv [B, L, 3 * 64 heads] bf16 -> out [B, L, 64 heads] bf16: per sample and head,
+    Softmax(Q K^T / 8) V."""
+    B, L, C3 = qkv.shape
+    C = 64 * heads
+    if C3 != 3 * C:
+        raise ValueError("qkv must be [B, L, 3 * 64 * heads]")
+    if out is None:
+        out = torch.empty(B, L, C, dtype=torch.bfloat16, device=qkv.device)
+    _check(lib().rs_attn_core(_ptr(qkv), B, L, int(heads), _ptr(out), _stream(stream)),
+           "rs_attn_core")
+    return out
+
+
+def rs_attn_sublayer(x: torch.Tensor, Wqkv, bqkv, Wo, bo, gamma, beta, heads: int,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x [B, L, C] bf16 -> x + SA(LN(x)) [B, L, C] bf16 (C = 64 heads)."""
+    B, L, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().rs_attn_sublayer(_ptr(x), B, L, C, int(heads), _ptr(Wqkv), _ptr(bqkv), _ptr(Wo),
+                                  _ptr(bo), _ptr(gamma), _ptr(beta), _ptr(out), _stream(stream)),
+           "rs_attn_sublayer")
+    return out
+
+
+def rs_attn_forward(x: torch.Tensor, Wqkv, bqkv, Wo, bo, gamma, beta, heads: int, keep_k: int,
+                    x_kept: Optional[torch.Tensor] = None,
+                    kept_idx: Optional[torch.Tensor] = None,
+                    scores: Optional[torch.Tensor] = None, stream=None, distance="l2",
+                    cls: bool = True) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """The attention sublayer, then pruning by its representation shift:
+    (x'_kept [B, n, C], kept_idx [B, n] int32, scores [B, L] fp32), n as in
+    rs_block_forward."""
+    B, L, C = x.shape
+    dev = x.device
+    n = keep_k + (1 if cls else 0)
+    if x_kept is None:
+        x_kept = torch.empty(B, n, C, dtype=torch.bfloat16, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(B, n, dtype=torch.int32, device=dev)
+    if scores is None:
+        scores = torch.empty(B, L, dtype=torch.float32, device=dev)
+    st = lib().rs_attn_forward_ex(_ptr(x), B, L, C, int(heads), _ptr(Wqkv), _ptr(bqkv), _ptr(Wo),
+                                  _ptr(bo), _ptr(gamma), _ptr(beta), int(keep_k), _dist(distance),
+                                  0 if cls else RS_NO_CLS, _ptr(x_kept), _ptr(kept_idx),
+                                  _ptr(scores), _stream(stream))
+    _check(st, "rs_attn_forward")
+    return x_kept, kept_idx, scores

@@ -112,6 +112,46 @@ int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W
                         int32_t* kept_idx, float* scores, void* stream);
 
 /*
+ * The attention sublayer that feeds the block (Eq. (5): x' = SA(LN(x)) + x) and
+ * that consumes its pruned output in the next layer. SA is Eq. (1),
+ * Softmax(Q K^T / sqrt(d)) V, in the multi-head form of the ViT models the paper
+ * runs: [Q, K, V] = LN(x) Wqkv^T + bqkv with Q, K, V at columns [0, C), [C, 2C),
+ * [2C, 3C) of the projection, heads of width d = 64 (head h at columns
+ * 64h .. 64h+63 of each), the heads' outputs concatenated, then the output
+ * projection Wo, bo. C = 64 * heads. The LayerNorm is the block's (biased
+ * variance, eps = 1e-6).
+ *   x     [B, L, C] bf16       the sublayer input
+ *   Wqkv  [3C, C], bqkv [3C]   bf16, nn.Linear layout
+ *   Wo    [C, C],  bo [C]      bf16
+ *   gamma, beta [C]            bf16, the sublayer's LayerNorm
+ * All device pointers, 16-byte aligned unless stated; workspace and error
+ * behaviour as for rs_block_forward (argument errors return before any launch).
+ */
+
+/* x_out [B, L, C] bf16 = x + SA(LN(x)). Four launches: LN statistics + weight
+ * fold, the QKV projection (the folded-LN tcgen05 GEMM without activation),
+ * rs_attn_core, the output projection with the residual (the fc2 GEMM, K = C). */
+int rs_attn_sublayer(const void* x, int B, int L, int C, int heads, const void* Wqkv,
+                     const void* bqkv, const void* Wo, const void* bo, const void* gamma,
+                     const void* beta, void* x_out, void* stream);
+
+/* rs_attn_sublayer followed by pruning on the representation shift through the
+ * attention, D(SA(LN(x)), x) (§3.3 "Operation choice" case (i)), with the
+ * distance and flags of rs_block_forward_ex: x_kept [B, n, C] bf16 holds the
+ * kept rows of x' (n = 1 + keep_k with a CLS token, keep_k with RS_NO_CLS),
+ * kept_idx [B, n] int32, scores [B, L] fp32 (4-byte aligned). */
+int rs_attn_forward_ex(const void* x, int B, int L, int C, int heads, const void* Wqkv,
+                       const void* bqkv, const void* Wo, const void* bo, const void* gamma,
+                       const void* beta, int keep_k, int distance, int flags, void* x_kept,
+                       int32_t* kept_idx, float* scores, void* stream);
+
+/* The attention core alone: out [B, L, 64 heads] bf16 = per sample and head,
+ * Softmax(Q K^T / 8) V from qkv [B, L, 3 * 64 heads] bf16 laid out as above (a
+ * tcgen05 kernel: scores and P V in TMEM, online softmax, one CTA per 128
+ * queries of a (sample, head)). 1 <= L <= RS_MAX_L, 64 heads <= RS_MAX_C. */
+int rs_attn_core(const void* qkv, int B, int L, int heads, void* out, void* stream);
+
+/*
  * Step-level entry points. rs_block_forward launches exactly these kernels in
  * this order; they are exported so that each step can be checked on its own.
  */

@@ -115,6 +115,45 @@ def test_extended_entry_points_argument_errors():
                                  None) == rs.RS_ERR_ALIGN
 
 
+def test_attention_entry_points_argument_errors():
+    lib = rs.lib()
+    w = FAKE
+
+    def sub(x=FAKE, B=2, L=197, C=384, heads=6, wt=w, out=FAKE):
+        return lib.rs_attn_sublayer(x, B, L, C, heads, wt, wt, wt, wt, wt, wt, out, None)
+
+    def fwd(B=2, L=197, C=384, heads=6, k=137, dist=0, flags=0, out=FAKE, idx=FAKE, sc=FAKE):
+        return lib.rs_attn_forward_ex(FAKE, B, L, C, heads, w, w, w, w, w, w, k, dist, flags,
+                                      out, idx, sc, None)
+
+    assert lib.rs_attn_core(FAKE, 0, 7, 2, FAKE, None) == rs.RS_OK     # empty batch
+    assert lib.rs_attn_core(None, 1, 7, 2, FAKE, None) == rs.RS_ERR_NULL
+    assert lib.rs_attn_core(FAKE, 1, 7, 2, None, None) == rs.RS_ERR_NULL
+    assert lib.rs_attn_core(MIS, 1, 7, 2, FAKE, None) == rs.RS_ERR_ALIGN
+    assert lib.rs_attn_core(FAKE, 1, 0, 2, FAKE, None) == rs.RS_ERR_SHAPE
+    assert lib.rs_attn_core(FAKE, 1, 7, 0, FAKE, None) == rs.RS_ERR_SHAPE
+    assert lib.rs_attn_core(FAKE, 1, 7, 33, FAKE, None) == rs.RS_ERR_SHAPE  # 64 * 33 > RS_MAX_C
+    assert lib.rs_attn_core(FAKE, 1, 16385, 2, FAKE, None) == rs.RS_ERR_SHAPE
+    assert sub(B=0) == rs.RS_OK
+    assert sub(C=384, heads=4) == rs.RS_ERR_SHAPE       # heads of width 64 only
+    assert sub(C=96, heads=1) == rs.RS_ERR_SHAPE
+    assert sub(x=None) == rs.RS_ERR_NULL
+    assert sub(wt=None) == rs.RS_ERR_NULL
+    assert sub(out=None) == rs.RS_ERR_NULL
+    assert sub(out=MIS) == rs.RS_ERR_ALIGN
+    assert sub(x=MIS) == rs.RS_ERR_ALIGN
+    assert fwd(B=0) == rs.RS_OK
+    assert fwd(k=197) == rs.RS_ERR_KEEP_K               # CLS kept: at most L - 1
+    assert fwd(k=198, flags=rs.RS_NO_CLS) == rs.RS_ERR_KEEP_K
+    assert fwd(k=-1) == rs.RS_ERR_KEEP_K
+    assert fwd(dist=3) == rs.RS_ERR_SHAPE
+    assert fwd(flags=2) == rs.RS_ERR_SHAPE
+    assert fwd(sc=None) == rs.RS_ERR_NULL
+    assert fwd(idx=None) == rs.RS_ERR_NULL
+    assert fwd(out=MIS) == rs.RS_ERR_ALIGN
+    assert fwd(heads=5) == rs.RS_ERR_SHAPE
+
+
 def test_library_has_no_torch_or_libcuda_link_dependency():
     out = os.popen(f"ldd {rs.LIB_PATH}").read()
     assert "libtorch" not in out and "libc10" not in out

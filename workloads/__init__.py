@@ -180,6 +180,42 @@ def random_block(B: int, L: int, C: int, H: int, seed: int, fg_rows: int = 0) ->
     return BlockInputs(x=x.to(torch.bfloat16), foreground=fg, weights=[draw_weights(g, C, H)])
 
 
+@dataclass
+class AttnWeights:
+    """The attention sublayer's parameters (nn.Linear layouts), bf16."""
+
+    Wqkv: torch.Tensor  # [3C, C]
+    bqkv: torch.Tensor  # [3C]
+    Wo: torch.Tensor    # [C, C]
+    bo: torch.Tensor    # [C]
+    gamma: torch.Tensor  # [C]
+    beta: torch.Tensor   # [C]
+
+
+def draw_attn_weights(C: int, seed: int, std: float = 0.02) -> AttnWeights:
+    """Attention sublayer weights from ``Generator(seed)`` in the order Wqkv, bqkv,
+    Wo, bo, gamma, beta: weights N(0, std) truncated at +-2 std (0.02 is the ViT
+    initialisation; larger values give peaked softmax rows), biases N(0, 0.01),
+    gamma = 1 + N(0, 0.05), beta ~ N(0, 0.02)."""
+    g = torch.Generator().manual_seed(seed)
+    Wqkv = _trunc_normal(g, (3 * C, C), std)
+    bqkv = torch.randn(3 * C, generator=g) * 0.01
+    Wo = _trunc_normal(g, (C, C), std)
+    bo = torch.randn(C, generator=g) * 0.01
+    gamma = 1.0 + torch.randn(C, generator=g) * 0.05
+    beta = torch.randn(C, generator=g) * 0.02
+    bf = torch.bfloat16
+    return AttnWeights(Wqkv.to(bf), bqkv.to(bf), Wo.to(bf), bo.to(bf), gamma.to(bf), beta.to(bf))
+
+
+def random_qkv(B: int, L: int, heads: int, seed: int, scale: float = 1.0) -> torch.Tensor:
+    """bf16 [B, L, 3 * 64 * heads] QKV projection values ~ N(0, scale^2): with head
+    width 64 and the 1/8 scaling, scale 1 gives scores of unit spread, scale 3
+    nearly one-hot softmax rows."""
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(B, L, 3 * 64 * heads, generator=g) * scale).to(torch.bfloat16)
+
+
 def random_partials(B: int, L: int, P: int, seed: int, ties: bool = False) -> torch.Tensor:
     """fp32 [B*L, P] non-negative per-row partial sums of squares (select-kernel inputs).
 
