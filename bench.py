@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -243,6 +244,52 @@ def time_attention(rs, wl, x_full, x_kept, peaks, dev, stream, reps: int):
     return res
 
 
+def deit_keep_schedule(L: int, depth: int = 12, layers=(1, 4, 7), ratio: float = 0.2):
+    """keep[l]: patch tokens kept after layer l (20% of the patch tokens pruned after
+    layers 1, 4 and 7, rounded to the nearest integer), -1 where a layer does not prune."""
+    keep = [-1] * depth
+    patches = L - 1
+    for l in layers:
+        patches -= int(math.floor(ratio * patches + 0.5))
+        keep[l] = patches
+    return keep
+
+
+def time_encoder_schedule(rs, wl, x, dev, stream, reps: int):
+    """A 12-layer encoder of this workload's width (attention sublayer + MLP per layer,
+    random ViT-initialised weights) through rs_encoder_forward, with the pruning
+    schedule of the DeiT runs and without pruning: images/s of each (mean of `reps`
+    calls between CUDA events, after two warm-up calls)."""
+    if reps <= 0 or wl.C % 64 or wl.stages != 1 or wl.L != 197:
+        return None
+    from workloads import draw_attn_weights, draw_weights
+    heads = wl.C // 64
+    layers = []
+    for l in range(12):
+        a = draw_attn_weights(wl.C, seed=2000 + l)
+        m = draw_weights(torch.Generator().manual_seed(3000 + l), wl.C, wl.H)
+        layers.append([t.to(dev) for t in (a.Wqkv, a.bqkv, a.Wo, a.bo, a.gamma, a.beta,
+                                           m.W1, m.b1, m.W2, m.b2, m.gamma, m.beta)])
+    res = {"depth": 12, "heads": heads, "batch": wl.B, "reps": reps,
+           "timing": "mean of back-to-back calls between CUDA events"}
+    for tag, keep in (("pruned", deit_keep_schedule(wl.L)), ("unpruned", [-1] * 12)):
+        for _ in range(2):
+            out = rs.rs_encoder_forward(x, layers, keep, heads, stream=stream)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            rs.rs_encoder_forward(x, layers, keep, heads, out=out, stream=stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / reps
+        res[tag] = {"keep": keep, "ms": ms, "images_per_s": wl.B / (ms / 1e3),
+                    "tokens_out": int(out.shape[1])}
+    assert rs.rs_get_last_device_error() == 0
+    res["speedup_pruned_vs_unpruned"] = res["unpruned"]["ms"] / res["pruned"]["ms"]
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -250,6 +297,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="deit_s", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--encoder-reps", type=int, default=5,
+                    help="calls per 12-layer encoder timing (0: skip that measurement)")
     ap.add_argument("--attn-reps", type=int, default=20,
                     help="calls per attention-sublayer timing (0: skip that measurement)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
@@ -506,6 +555,7 @@ def main():
     clocks.stop()
 
     attn = time_attention(rs, wl, x, outs[0][0], peaks, dev, stream, args.attn_reps)
+    sched = time_encoder_schedule(rs, wl, x, dev, stream, args.encoder_reps)
 
     cpu = None
     if rank == 0 and args.cpu_budget > 0:
@@ -550,6 +600,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (own streams)"},
         "attention_next_layer": attn,
+        "encoder_schedule": sched,
         "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

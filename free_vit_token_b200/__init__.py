@@ -15,6 +15,7 @@ from .rs import (  # noqa: F401
     rs_attn_forward,
     rs_attn_sublayer,
     rs_block_forward,
+    rs_encoder_forward,
     rs_fc2_residual_shift,
     rs_debug_fc1_skip_load,
     rs_fc1_gelu_folded,
@@ -26,6 +27,7 @@ from .rs import (  # noqa: F401
     rs_ln_fc1_gelu_noalloc,
     rs_ln_fc1_gelu_staged,
     rs_ln_stats,
+    rs_mlp_forward,
     rs_num_partials,
     rs_release_workspace,
     rs_select_gather,

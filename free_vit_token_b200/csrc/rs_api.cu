@@ -20,6 +20,8 @@ constexpr int kMaxDevices = 64;
 struct DevState {
   void* ws = nullptr;
   size_t ws_bytes = 0;
+  void* act = nullptr;  // rs_encoder_forward: activations between layers
+  size_t act_bytes = 0;
   int* err = nullptr;  // device status flag (one int)
   int num_sms = 0;
 };
@@ -286,15 +288,15 @@ AttnWs attn_ws_layout(int64_t M, int C) {
   return a;
 }
 
-// The QKV projection [B*L, 3C] as a [B][L][3C] tensor with {64, 128, 1} boxes.
-int make_tmap_qkv(CUtensorMap* m, const void* qkv, int B, int L, int C) {
+// The QKV projection [B*L, 3C] as a [B][L][3C] tensor with {64, box_rows, 1} boxes.
+int make_tmap_qkv(CUtensorMap* m, const void* qkv, int B, int L, int C, int box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return RS_ERR_CUDA;
   const cuuint64_t row = static_cast<cuuint64_t>(3 * C) * 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * C), static_cast<cuuint64_t>(L),
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[2] = {row, row * static_cast<cuuint64_t>(L)};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -310,8 +312,9 @@ int check_heads(int C, int heads) {
 
 int run_attn_core(DevState& st, const void* qkv, int B, int L, int C, int heads, void* out,
                   cudaStream_t s, bool pdl) {
-  CUtensorMap tm;
-  RS_TRY(make_tmap_qkv(&tm, qkv, B, L, C));
+  CUtensorMap tmQ, tmKV;
+  RS_TRY(make_tmap_qkv(&tmQ, qkv, B, L, C, rs::attn_q_box_rows()));
+  RS_TRY(make_tmap_qkv(&tmKV, qkv, B, L, C, rs::attn_kv_box_rows()));
   rs::AttnParams p{};
   p.B = B;
   p.L = L;
@@ -320,7 +323,7 @@ int run_attn_core(DevState& st, const void* qkv, int B, int L, int C, int heads,
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
-  RS_CUDA(rs::launch_attn(tm, p, s, pdl));
+  RS_CUDA(rs::launch_attn(tmQ, tmKV, p, s, pdl));
   return RS_OK;
 }
 
@@ -347,6 +350,59 @@ int run_attn_sublayer(DevState& st, const void* x, int B, int L, int C, int head
                  /*pdl=*/true));
   if (ws_out) *ws_out = ws;
   if (w_out) *w_out = w;
+  return RS_OK;
+}
+
+// The pruned MLP block (rs_block_forward_ex's launches) on validated arguments.
+int run_block(DevState& st, const void* x, int B, int L, int C, int H, const void* W1,
+              const void* b1, const void* W2, const void* b2, const void* gamma,
+              const void* beta, int keep_k, int distance, int flags, void* y_kept,
+              int32_t* kept_idx, float* scores, cudaStream_t s) {
+  const int M = B * L;
+  const WsLayout w = ws_layout(M, C, H);
+  RS_TRY(ensure_ws(st, w.total));
+  uint8_t* ws = static_cast<uint8_t*>(st.ws);
+  void* hidden = ws + w.hidden;
+  void* y = ws + w.y;
+  float* partials = reinterpret_cast<float*>(ws + w.partials);
+  const int np =
+      rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
+  RS_TRY(run_fc1(st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
+  RS_TRY(run_fc2(st, hidden, x, M, C, H, W2, b2, y, partials, distance, s, /*pdl=*/true));
+  RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, distance,
+                                   !(flags & RS_NO_CLS), scores, kept_idx, y_kept, st.num_sms, s,
+                                   /*pdl=*/true));
+  return RS_OK;
+}
+
+// The non-pruning MLP sublayer (rs_mlp_forward's launches) on validated arguments.
+int run_mlp(DevState& st, const void* x, int M, int C, int H, const void* W1, const void* b1,
+            const void* W2, const void* b2, const void* gamma, const void* beta, void* y,
+            cudaStream_t s) {
+  const WsLayout w = ws_layout(M, C, H);
+  RS_TRY(ensure_ws(st, w.total));
+  uint8_t* ws = static_cast<uint8_t*>(st.ws);
+  void* hidden = ws + w.hidden;
+  RS_TRY(run_fc1(st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
+  RS_TRY(run_fc2(st, hidden, x, M, C, H, W2, b2, y, reinterpret_cast<float*>(ws + w.partials),
+                 RS_DIST_L2, s, /*pdl=*/true));
+  return RS_OK;
+}
+
+// Caller holds g_mu; grows the encoder's activation buffer (stream-ordered use).
+int ensure_act(DevState& st, size_t bytes) {
+  if (st.act_bytes >= bytes) return RS_OK;
+  if (st.act != nullptr) {
+    cudaDeviceSynchronize();
+    cudaFree(st.act);
+    st.act = nullptr;
+    st.act_bytes = 0;
+  }
+  if (cudaMalloc(&st.act, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return RS_ERR_NO_MEM;
+  }
+  st.act_bytes = bytes;
   return RS_OK;
 }
 
@@ -433,6 +489,24 @@ static int ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const
 int rs_ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const void* b1,
                    const void* gamma, const void* beta, void* hidden, void* stream) {
   return ln_fc1_gelu(x, M, C, H, W1, b1, gamma, beta, hidden, false, stream);
+}
+
+int rs_mlp_forward(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                   const void* W2, const void* b2, const void* gamma, const void* beta, void* y,
+                   void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (M == 0) return RS_OK;
+  if (!x || !W1 || !b1 || !W2 || !b2 || !gamma || !beta || !y) return RS_ERR_NULL;
+  if (!al16(x) || !al16(W1) || !al16(b1) || !al16(W2) || !al16(b2) || !al16(gamma) ||
+      !al16(beta) || !al16(y))
+    return RS_ERR_ALIGN;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_mlp(*st, x, M, C, H, W1, b1, W2, b2, gamma, beta, y, s);
 }
 
 int rs_ln_fc1_gelu_staged(const void* x, int M, int C, int H, const void* W1, const void* b1,
@@ -669,27 +743,13 @@ int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W
   if (!al16(x) || !al16(W1) || !al16(b1) || !al16(W2) || !al16(b2) || !al16(gamma) ||
       !al16(beta) || !al16(y_kept) || !al4(kept_idx) || !al4(scores))
     return RS_ERR_ALIGN;
-  const int M = static_cast<int>(M64);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   std::lock_guard<std::mutex> lock(g_mu);
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
-  const WsLayout w = ws_layout(M, C, H);
-  RS_TRY(ensure_ws(*st, w.total));
-  uint8_t* ws = static_cast<uint8_t*>(st->ws);
-  void* hidden = ws + w.hidden;
-  void* y = ws + w.y;
-  float* partials = reinterpret_cast<float*>(ws + w.partials);
-  const int np =
-      rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
-
-  RS_TRY(run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
-  RS_TRY(run_fc2(*st, hidden, x, M, C, H, W2, b2, y, partials, distance, s, /*pdl=*/true));
-  RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, distance,
-                                   !(flags & RS_NO_CLS), scores, kept_idx, y_kept, st->num_sms, s,
-                                   /*pdl=*/true));
-  return RS_OK;
+  return run_block(*st, x, B, L, C, H, W1, b1, W2, b2, gamma, beta, keep_k, distance, flags,
+                   y_kept, kept_idx, scores, s);
 }
 int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, const void* b1,
                      const void* W2, const void* b2, const void* gamma, const void* beta,
@@ -753,6 +813,66 @@ int rs_attn_forward_ex(const void* x, int B, int L, int C, int heads, const void
   return RS_OK;
 }
 
+int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int depth,
+                       const void* const* weights, const int* keep, void* out, void* stream) {
+  if (B < 0 || L < 1 || L > RS_MAX_L || depth < 1 || depth > 1024) return RS_ERR_SHAPE;
+  RS_TRY(check_heads(C, heads));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, H > 3 * C ? H : 3 * C));
+  if (!weights || !keep) return RS_ERR_NULL;
+  int Lc = L;
+  for (int l = 0; l < depth; ++l) {
+    if (keep[l] >= 0) {
+      RS_TRY(check_keep(keep[l], Lc, 0));
+      Lc = 1 + keep[l];
+    }
+  }
+  if (B == 0) return RS_OK;
+  if (!x || !out) return RS_ERR_NULL;
+  if (!al16(x) || !al16(out)) return RS_ERR_ALIGN;
+  for (int i = 0; i < 12 * depth; ++i) {
+    if (!weights[i]) return RS_ERR_NULL;
+    if (!al16(weights[i])) return RS_ERR_ALIGN;
+  }
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  // activations: x' and two ping-pong layer outputs [B, L, C] bf16, then the
+  // kept indices and scores of a pruning layer
+  const size_t xb = align_up(static_cast<size_t>(B) * L * C * 2, 1024);
+  const size_t ib = align_up(static_cast<size_t>(B) * L * 4, 1024);
+  RS_TRY(ensure_act(*st, 3 * xb + 2 * ib));
+  uint8_t* act = static_cast<uint8_t*>(st->act);
+  void* xp = act;
+  void* buf[2] = {act + xb, act + 2 * xb};
+  int32_t* kept = reinterpret_cast<int32_t*>(act + 3 * xb);
+  float* scores = reinterpret_cast<float*>(act + 3 * xb + ib);
+  // the largest workspace any layer needs, once, before the first launch
+  {
+    const int64_t M = static_cast<int64_t>(B) * L;
+    const size_t a = attn_ws_layout(M, C).w.total, m = ws_layout(M, C, H).total;
+    RS_TRY(ensure_ws(*st, a > m ? a : m));
+  }
+  const void* cur = x;
+  Lc = L;
+  for (int l = 0; l < depth; ++l) {
+    const void* const* w = weights + 12 * l;
+    void* nxt = l + 1 == depth ? out : buf[l & 1];
+    RS_TRY(run_attn_sublayer(*st, cur, B, Lc, C, heads, w[0], w[1], w[2], w[3], w[4], w[5], xp,
+                             RS_DIST_L2, s, nullptr, nullptr));
+    if (keep[l] >= 0) {
+      RS_TRY(run_block(*st, xp, B, Lc, C, H, w[6], w[7], w[8], w[9], w[10], w[11], keep[l],
+                       RS_DIST_L2, 0, nxt, kept, scores, s));
+      Lc = 1 + keep[l];
+    } else {
+      RS_TRY(run_mlp(*st, xp, B * Lc, C, H, w[6], w[7], w[8], w[9], w[10], w[11], nxt, s));
+    }
+    cur = nxt;
+  }
+  return RS_OK;
+}
+
 int rs_get_last_device_error(void* stream) {
   std::lock_guard<std::mutex> lock(g_mu);
   DevState* st = nullptr;
@@ -773,13 +893,16 @@ void rs_release_workspace(void) {
   if (cudaGetDevice(&cur) != cudaSuccess) return;
   for (int d = 0; d < kMaxDevices; ++d) {
     DevState& st = g_dev[d];
-    if (st.ws == nullptr) continue;
+    if (st.ws == nullptr && st.act == nullptr) continue;
     if (cudaSetDevice(d) == cudaSuccess) {
       cudaDeviceSynchronize();
-      cudaFree(st.ws);
+      if (st.ws) cudaFree(st.ws);
+      if (st.act) cudaFree(st.act);
     }
     st.ws = nullptr;
     st.ws_bytes = 0;
+    st.act = nullptr;
+    st.act_bytes = 0;
   }
   cudaSetDevice(cur);
 }

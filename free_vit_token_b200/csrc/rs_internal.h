@@ -143,8 +143,9 @@ cudaError_t launch_select_gather(const float* partials, int num_partials, const 
 
 // Attention core (rs_attn.cu): per sample and head of width 64, Softmax(Q K^T / 8) V
 // from a QKV projection [B, L, 3C] (Q, K, V at columns 0, C, 2C; head h at +64 h),
-// written to out [B, L, C] (head h at columns 64 h). The tensor map views the QKV
-// buffer as [B][L][3C] with {64, 128, 1} boxes and the 128-byte swizzle.
+// written to out [B, L, C] (head h at columns 64 h). Both tensor maps view the
+// QKV buffer as [B][L][3C] with the 128-byte swizzle, in boxes of {64,
+// attn_q_box_rows(), 1} (Q) and {64, attn_kv_box_rows(), 1} (K and V).
 struct AttnParams {
   int B, L, C, heads;
   __nv_bfloat16* out;
@@ -152,7 +153,9 @@ struct AttnParams {
   unsigned long long timeout_ns;  // limit of one pipeline wait
 };
 size_t attn_smem_bytes();
-cudaError_t launch_attn(const CUtensorMap& tmQKV, const AttnParams& p, cudaStream_t stream,
-                        bool pdl = false);
+int attn_q_box_rows();
+int attn_kv_box_rows();
+cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
+                        cudaStream_t stream, bool pdl = false);
 
 }  // namespace rs

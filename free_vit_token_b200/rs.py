@@ -47,7 +47,10 @@ SIGNATURES = {
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
     "rs_select_gather": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
+    "rs_mlp_forward": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_attn_core": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "rs_encoder_forward": (_i, [_vp, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp),
+                                ctypes.POINTER(_i), _vp, _vp]),
     "rs_attn_sublayer": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_attn_forward_ex": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
                                 _vp, _ip, _fp, _vp]),
@@ -363,3 +366,42 @@ def rs_attn_forward(x: torch.Tensor, Wqkv, bqkv, Wo, bo, gamma, beta, heads: int
                                   _ptr(scores), _stream(stream))
     _check(st, "rs_attn_forward")
     return x_kept, kept_idx, scores
+
+
+def rs_mlp_forward(x: torch.Tensor, W1, b1, W2, b2, gamma, beta,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x [..., C] bf16 -> x + MLP(LN(x)) (no scoring, no pruning), same shape."""
+    C = x.shape[-1]
+    M = x.numel() // C
+    H = W1.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().rs_mlp_forward(_ptr(x), M, C, H, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                                _ptr(gamma), _ptr(beta), _ptr(out), _stream(stream)),
+           "rs_mlp_forward")
+    return out
+
+
+ENCODER_WEIGHT_ORDER = ("Wqkv", "bqkv", "Wo", "bo", "gamma1", "beta1",
+                        "W1", "b1", "W2", "b2", "gamma2", "beta2")
+
+
+def rs_encoder_forward(x: torch.Tensor, layers, keep, heads: int,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x [B, L, C] bf16 through len(layers) encoder layers; `layers[l]` is a sequence
+    of the 12 weight tensors in ENCODER_WEIGHT_ORDER, keep[l] the patch tokens kept
+    after layer l (negative: no pruning). Returns [B, L_out, C]."""
+    B, L, C = x.shape
+    depth = len(layers)
+    H = layers[0][6].shape[0]
+    ptrs = (_vp * (12 * depth))(*[_ptr(t) for lw in layers for t in lw])
+    kk = (_i * depth)(*[int(k) for k in keep])
+    L_out = L
+    for k in keep:
+        if k >= 0:
+            L_out = 1 + int(k)
+    if out is None:
+        out = torch.empty(B, L_out, C, dtype=torch.bfloat16, device=x.device)
+    _check(lib().rs_encoder_forward(_ptr(x), B, L, C, H, int(heads), depth, ptrs, kk, _ptr(out),
+                                    _stream(stream)), "rs_encoder_forward")
+    return out

@@ -111,6 +111,14 @@ int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W
                         const void* beta, int keep_k, int distance, int flags, void* y_kept,
                         int32_t* kept_idx, float* scores, void* stream);
 
+/* The MLP sublayer without pruning, y = x + MLP(LN(x)) (Eq. (6)), as the layers
+ * of a pruning schedule that do not prune run it: the same three launches as the
+ * first three of rs_block_forward (LN statistics + fold, fc1, fc2), y written to
+ * the caller's buffer. x, y [M, C] bf16; weights as for rs_block_forward. */
+int rs_mlp_forward(const void* x, int M, int C, int H, const void* W1, const void* b1,
+                   const void* W2, const void* b2, const void* gamma, const void* beta, void* y,
+                   void* stream);
+
 /*
  * The attention sublayer that feeds the block (Eq. (5): x' = SA(LN(x)) + x) and
  * that consumes its pruned output in the next layer. SA is Eq. (1),
@@ -144,6 +152,26 @@ int rs_attn_forward_ex(const void* x, int B, int L, int C, int heads, const void
                        const void* bqkv, const void* Wo, const void* bo, const void* gamma,
                        const void* beta, int keep_k, int distance, int flags, void* x_kept,
                        int32_t* kept_idx, float* scores, void* stream);
+
+/* A ViT encoder of `depth` layers, each the attention sublayer (Eq. (5)) then the
+ * MLP sublayer (Eq. (6)), with representation-shift pruning (L2 shift through the
+ * MLP, CLS kept) after the MLP of the layers that keep[l] >= 0 names: those keep
+ * keep[l] patch tokens (0 <= keep[l] <= tokens entering layer l - 1); keep[l] < 0
+ * runs the MLP without pruning (rs_mlp_forward). The pruning schedule of the
+ * paper's DeiT runs (§4.2) keeps 80% of the tokens after layers 1, 4 and 7.
+ *   x        [B, L, C] bf16, the first layer's input
+ *   weights  12 * depth device pointers, per layer: Wqkv, bqkv, Wo, bo, gamma1,
+ *            beta1 (attention sublayer), W1, b1, W2, b2, gamma2, beta2 (MLP), all
+ *            bf16, 16-byte aligned, shapes as for rs_attn_sublayer and
+ *            rs_block_forward (H = hidden width)
+ *   keep     depth ints (host memory)
+ *   out      [B, L_out, C] bf16, L_out = 1 + the last keep[l] >= 0, else L
+ * The library holds the activations between layers (three [B, L, C] buffers and
+ * one layer's kept indices and scores) in a cached device buffer beside the
+ * workspace; rs_release_workspace frees both. Argument errors (any layer's)
+ * return before the first launch. */
+int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int depth,
+                       const void* const* weights, const int* keep, void* out, void* stream);
 
 /* The attention core alone: out [B, L, 64 heads] bf16 = per sample and head,
  * Softmax(Q K^T / 8) V from qkv [B, L, 3 * 64 heads] bf16 laid out as above (a

@@ -154,6 +154,40 @@ def test_attention_entry_points_argument_errors():
     assert fwd(heads=5) == rs.RS_ERR_SHAPE
 
 
+def test_encoder_and_mlp_entry_points_argument_errors():
+    lib = rs.lib()
+    depth = 3
+    good = (ctypes.c_void_p * (12 * depth))(*([FAKE] * (12 * depth)))
+    holes = (ctypes.c_void_p * (12 * depth))(*([FAKE] * (12 * depth - 1) + [None]))
+    mis = (ctypes.c_void_p * (12 * depth))(*([FAKE] * 5 + [MIS] + [FAKE] * (12 * depth - 6)))
+
+    def keep(*k):
+        return (ctypes.c_int * depth)(*k)
+
+    def enc(x=FAKE, B=2, L=197, C=384, H=1536, heads=6, w=good, k=None, out=FAKE, d=depth):
+        return lib.rs_encoder_forward(x, B, L, C, H, heads, d, w,
+                                      k if k is not None else keep(-1, 157, -1), out, None)
+
+    assert enc(B=0) == rs.RS_OK
+    assert enc(x=None) == rs.RS_ERR_NULL
+    assert enc(out=None) == rs.RS_ERR_NULL
+    assert enc(w=holes) == rs.RS_ERR_NULL
+    assert enc(w=mis) == rs.RS_ERR_ALIGN
+    assert enc(heads=5) == rs.RS_ERR_SHAPE
+    assert enc(H=100) == rs.RS_ERR_SHAPE
+    assert enc(d=0) == rs.RS_ERR_SHAPE
+    assert enc(k=keep(-1, 197, -1)) == rs.RS_ERR_KEEP_K        # more than L - 1 patches
+    assert enc(k=keep(100, 101, -1)) == rs.RS_ERR_KEEP_K       # later layer keeps more
+    assert lib.rs_mlp_forward(FAKE, 0, 384, 1536, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              None) == rs.RS_OK
+    assert lib.rs_mlp_forward(FAKE, 10, 384, 1536, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                              None) == rs.RS_ERR_NULL
+    assert lib.rs_mlp_forward(FAKE, 10, 100, 1536, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              None) == rs.RS_ERR_SHAPE
+    assert lib.rs_mlp_forward(MIS, 10, 384, 1536, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              None) == rs.RS_ERR_ALIGN
+
+
 def test_library_has_no_torch_or_libcuda_link_dependency():
     out = os.popen(f"ldd {rs.LIB_PATH}").read()
     assert "libtorch" not in out and "libc10" not in out
