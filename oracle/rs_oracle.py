@@ -142,6 +142,23 @@ def block_forward(x, W1, b1, W2, b2, gamma, beta, keep_k: int, eps: float = EPS,
     return y_kept, kept, s, y
 
 
+def block_shift_forward(x_in, x, W1, b1, W2, b2, gamma, beta, keep_k: int, eps: float = EPS,
+                        metric: str = "l2", cls: bool = True):
+    """Pruning on the shift through the entire attention block, §3.3 "Operation
+    choice" case (iii): s = D(x-hat, x_in), with x-hat = y = x' + MLP(LN(x')) the
+    block output (Eq. (6)) and x_in the block input that Eq. (5) started from.
+    x_in, x (= x') [B, L, C]; returns what block_forward returns."""
+    x_in = np.asarray(x_in, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    B, L, C = x.shape
+    _, y, _ = sublayer(x.reshape(B * L, C), W1, b1, W2, b2, gamma, beta, eps, metric)
+    s = shift_score(y, x_in.reshape(B * L, C), metric).reshape(B, L)
+    y = y.reshape(B, L, C)
+    kept = np.stack([select_topk(s[b], keep_k, cls) for b in range(B)])
+    y_kept = np.stack([gather(y[b], kept[b]) for b in range(B)])
+    return y_kept, kept, s, y
+
+
 def finalize_scores_f32(partials: np.ndarray, B: int, L: int, metric: str = "l2") -> np.ndarray:
     """Scores from fp32 per-row partial sums, in fp32 (correctly rounded operations).
 

@@ -340,6 +340,36 @@ def pin_finalize_f32(o):
     assert np.allclose(f(p, 1, 40, "cosine")[0], ref, rtol=0, atol=1e-6)
 
 
+def pin_block_shift(o):
+    """The whole-block shift D(y, x_in) (§3.3 case (iii)). With W2 = 0, b2 = 0 the MLP
+    adds nothing, y = x', and the shift is D(x', x_in): built here as x_in = x' - delta
+    with rows of known size, so s_l2 = ||delta||, s_l1 = sum |delta| and pruning keeps
+    the largest deltas. With x_in = x' and b2 = c the shift is ||h|| = ||c|| for every
+    token: all scores tie and the lowest indices are kept."""
+    rng = np.random.default_rng(22)
+    C, H, L = 8, 16, 7
+    w = _rng_weights(rng, C, H)
+    w["W2"] = np.zeros((C, H))
+    w["b2"] = np.zeros(C)
+    xp = rng.normal(0, 1, (1, L, C))
+    sizes = np.array([0.5, 2.0, 0.25, 3.0, 1.0, 4.0, 1.5])
+    d = rng.normal(0, 1, (L, C))
+    delta = d / np.linalg.norm(d, axis=1, keepdims=True) * sizes[:, None]
+    x_in = xp - delta[None]
+    for metric in ("l2", "l1"):
+        yk, kept, s, y = o.block_shift_forward(x_in, xp, keep_k=3, metric=metric, **w)
+        assert np.array_equal(y, xp)
+        want = sizes if metric == "l2" else np.abs(delta).sum(axis=1)
+        assert np.allclose(s[0], want, atol=1e-12, rtol=0), (metric, s)
+    _, kept, _, _ = o.block_shift_forward(x_in, xp, keep_k=3, **w)
+    assert kept[0].tolist() == [0, 1, 3, 5]          # CLS, then sizes 2.0, 3.0, 4.0
+    c = rng.normal(0, 1, C)
+    w["b2"] = c
+    _, kept, s, y = o.block_shift_forward(xp, xp, keep_k=3, **w)
+    assert np.allclose(s[0], np.linalg.norm(c), atol=1e-12, rtol=0)
+    assert kept[0].tolist() == [0, 1, 2, 3]
+
+
 def pin_gather(o):
     """The kept rows of y, in kept order."""
     rng = np.random.default_rng(18)
@@ -350,6 +380,7 @@ def pin_gather(o):
 
 ALL_PINS = [
     pin_gelu_table,
+    pin_block_shift,
     pin_metrics_hand_example,
     pin_metric_invariants,
     pin_topk_no_cls_exhaustive,

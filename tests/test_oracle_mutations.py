@@ -175,7 +175,30 @@ def _finalize_l1_sqrt(partials, B, L, metric="l2"):
     return orig["finalize_scores_f32"](partials, B, L, "l2")
 
 
+def _block_shift_vs_x_prime(x_in, x, W1, b1, W2, b2, gamma, beta, keep_k, eps=rs_oracle.EPS,
+                            metric="l2", cls=True):
+    # compares y with x' instead of the block input: the MLP shift of case (ii) in disguise
+    return _orig_block_shift(x, x, W1, b1, W2, b2, gamma, beta, keep_k, eps, metric, cls)
+
+
+def _block_shift_of_h(x_in, x, W1, b1, W2, b2, gamma, beta, keep_k, eps=rs_oracle.EPS,
+                      metric="l2", cls=True):
+    # compares the MLP output h (not the block output y) with the block input
+    x_in = np.asarray(x_in, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    B, L, C = x.shape
+    h, y, _ = rs_oracle.sublayer(x.reshape(B * L, C), W1, b1, W2, b2, gamma, beta, eps, metric)
+    s = rs_oracle.shift_score(h, x_in.reshape(B * L, C), metric).reshape(B, L)
+    y = y.reshape(B, L, C)
+    kept = np.stack([rs_oracle.select_topk(s[b], keep_k, cls) for b in range(B)])
+    return np.stack([y[b][kept[b]] for b in range(B)]), kept, s, y
+
+
+_orig_block_shift = rs_oracle.block_shift_forward
+
 MUTATIONS = {
+    "block_shift_against_x_prime": ("block_shift_forward", _block_shift_vs_x_prime),
+    "block_shift_of_mlp_output": ("block_shift_forward", _block_shift_of_h),
     "ln_unbiased_var": ("layer_norm", _ln_unbiased),
     "ln_drops_beta": ("layer_norm", _ln_no_beta),
     "ln_drops_gamma": ("layer_norm", _ln_no_gamma),
