@@ -15,6 +15,7 @@ from .rs import (  # noqa: F401
     rs_attn_forward,
     rs_attn_sublayer,
     rs_block_forward,
+    rs_block_forward_block_shift,
     rs_encoder_forward,
     rs_fc2_residual_shift,
     rs_debug_fc1_skip_load,

@@ -207,7 +207,8 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
 }
 
 int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H, const void* W2,
-            const void* b2, void* y, float* partials, int dist, cudaStream_t s, bool pdl = false) {
+            const void* b2, void* y, float* partials, int dist, cudaStream_t s, bool pdl = false,
+            const void* shift_ref = nullptr) {
   const int bn = rs::fc2_block_n(C);
   const bool pair = rs::gemm_pair(M, H, false);
   CUtensorMap tmH, tmW, tmY;
@@ -225,6 +226,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   p.resid = static_cast<const __nv_bfloat16*>(x);
   p.partials = partials;
   p.dist = dist;
+  p.shift_ref = static_cast<const __nv_bfloat16*>(shift_ref);
   p.num_partials = rs::dist_partials(dist) * rs::kFc2PartialsPerTile * p.n_blocks;
   p.err = st.err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
@@ -357,7 +359,8 @@ int run_attn_sublayer(DevState& st, const void* x, int B, int L, int C, int head
 int run_block(DevState& st, const void* x, int B, int L, int C, int H, const void* W1,
               const void* b1, const void* W2, const void* b2, const void* gamma,
               const void* beta, int keep_k, int distance, int flags, void* y_kept,
-              int32_t* kept_idx, float* scores, cudaStream_t s) {
+              int32_t* kept_idx, float* scores, cudaStream_t s,
+              const void* shift_ref = nullptr) {
   const int M = B * L;
   const WsLayout w = ws_layout(M, C, H);
   RS_TRY(ensure_ws(st, w.total));
@@ -368,7 +371,8 @@ int run_block(DevState& st, const void* x, int B, int L, int C, int H, const voi
   const int np =
       rs::dist_partials(distance) * rs::kFc2PartialsPerTile * C / rs::fc2_block_n(C);
   RS_TRY(run_fc1(st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
-  RS_TRY(run_fc2(st, hidden, x, M, C, H, W2, b2, y, partials, distance, s, /*pdl=*/true));
+  RS_TRY(run_fc2(st, hidden, x, M, C, H, W2, b2, y, partials, distance, s, /*pdl=*/true,
+                 shift_ref));
   RS_CUDA(rs::launch_select_gather(partials, np, y, B, L, C, keep_k, distance,
                                    !(flags & RS_NO_CLS), scores, kept_idx, y_kept, st.num_sms, s,
                                    /*pdl=*/true));
@@ -751,6 +755,34 @@ int rs_block_forward_ex(const void* x, int B, int L, int C, int H, const void* W
   return run_block(*st, x, B, L, C, H, W1, b1, W2, b2, gamma, beta, keep_k, distance, flags,
                    y_kept, kept_idx, scores, s);
 }
+int rs_block_forward_block_shift_ex(const void* x_in, const void* x, int B, int L, int C, int H,
+                                    const void* W1, const void* b1, const void* W2,
+                                    const void* b2, const void* gamma, const void* beta,
+                                    int keep_k, int distance, int flags, void* y_kept,
+                                    int32_t* kept_idx, float* scores, void* stream) {
+  if (B > 0 && !x_in) return RS_ERR_NULL;
+  if (!al16(x_in)) return RS_ERR_ALIGN;
+  RS_TRY(check_mode(distance, flags));
+  if (B < 0 || L < 1 || L > RS_MAX_L) return RS_ERR_SHAPE;
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, H));
+  RS_TRY(check_keep(keep_k, L, flags));
+  if (B == 0) return RS_OK;
+  const bool rows_out = keep_k + !(flags & RS_NO_CLS) > 0;
+  if (!x || !W1 || !b1 || !W2 || !b2 || !gamma || !beta || !scores ||
+      (rows_out && (!y_kept || !kept_idx)))
+    return RS_ERR_NULL;
+  if (!al16(x) || !al16(W1) || !al16(b1) || !al16(W2) || !al16(b2) || !al16(gamma) ||
+      !al16(beta) || !al16(y_kept) || !al4(kept_idx) || !al4(scores))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_block(*st, x, B, L, C, H, W1, b1, W2, b2, gamma, beta, keep_k, distance, flags,
+                   y_kept, kept_idx, scores, static_cast<cudaStream_t>(stream), x_in);
+}
+
 int rs_block_forward(const void* x, int B, int L, int C, int H, const void* W1, const void* b1,
                      const void* W2, const void* b2, const void* gamma, const void* beta,
                      int keep_k, void* y_kept, int32_t* kept_idx, float* scores, void* stream) {

@@ -88,6 +88,8 @@ struct MlpParams {
                                   // first tile (-1: off)
   int dist;                       // fc2: kDistL2, kDistL1 or kDistCos
   int linear;                     // folded-LN fc1: 0 = erf-GELU, 1 = no activation (QKV)
+  const __nv_bfloat16* shift_ref; // fc2: null, or [M, N]: the shift compares y = x' + h with
+                                  // this block input instead of h with x' (§3.3 case (iii))
 };
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);

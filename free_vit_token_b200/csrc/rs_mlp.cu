@@ -456,13 +456,22 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
       }
       const uint4* xrow =
           reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.N + col0);
+      // whole-block shift (§3.3 case (iii)): the distance compares y = x' + h with
+      // the block input at p.shift_ref instead of h with x'
+      const bool has_ref = EPI == kEpiResidShift && p.shift_ref != nullptr;
+      const uint4* zrow =
+          reinterpret_cast<const uint4*>(p.shift_ref + static_cast<size_t>(row) * p.N + col0);
       uint32_t ra[16], rb[16];
-      uint4 xa[2] = {}, xb[2] = {};
+      uint4 xa[2] = {}, xb[2] = {}, za[2] = {}, zb[2] = {};
       tmem_ld16_async(t_row, ra);
       if constexpr (EPI == kEpiResidShift) {
         if (row_ok) {
           xa[0] = __ldg(xrow);
           xa[1] = __ldg(xrow + 1);
+          if (has_ref) {
+            za[0] = __ldg(zrow);
+            za[1] = __ldg(zrow + 1);
+          }
         }
       }
 #pragma unroll
@@ -471,6 +480,8 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
         uint32_t(&nx)[16] = (n & 1) ? ra : rb;
         uint4(&xv)[2] = (n & 1) ? xb : xa;
         uint4(&xn)[2] = (n & 1) ? xa : xb;
+        uint4(&zv)[2] = (n & 1) ? zb : za;
+        uint4(&zn)[2] = (n & 1) ? za : zb;
         tmem_wait_ld();
         reg_fence16(r);
         if (n + 1 < NCH) {
@@ -479,6 +490,10 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
             if (row_ok) {
               xn[0] = __ldg(xrow + (n + 1) * 2);
               xn[1] = __ldg(xrow + (n + 1) * 2 + 1);
+              if (has_ref) {
+                zn[0] = __ldg(zrow + (n + 1) * 2);
+                zn[1] = __ldg(zrow + (n + 1) * 2 + 1);
+              }
             }
           }
         } else {
@@ -548,43 +563,44 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
             }
           } else {
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
-            // h in fp32 before rounding; the distance is uniform over the launch
+            const uint32_t* zw = reinterpret_cast<const uint32_t*>(zv);
+            // h in fp32 before rounding; the distance compares (f, g) = (h, x') or, for
+            // the whole-block shift, (x' + h, block input). Uniform over the launch.
+#define RS_SHIFT_OPERANDS(e)                                              \
+  const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);                     \
+  const float h0 = __uint_as_float(r[2 * (e)]) + bf16lo(bw[e]);           \
+  const float h1 = __uint_as_float(r[2 * (e) + 1]) + bf16hi(bw[e]);       \
+  outw[e] = pack_bf16x2(x0 + h0, x1 + h1);                                \
+  const float f0 = has_ref ? x0 + h0 : h0, f1 = has_ref ? x1 + h1 : h1;   \
+  const float g0 = has_ref ? bf16lo(zw[e]) : x0, g1 = has_ref ? bf16hi(zw[e]) : x1;
             if (p.dist == kDistCos) {
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
-                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
-                c_hx = fmaf(h0, x0, c_hx);
-                c_hx = fmaf(h1, x1, c_hx);
-                c_hh = fmaf(h0, h0, c_hh);
-                c_hh = fmaf(h1, h1, c_hh);
-                c_xx = fmaf(x0, x0, c_xx);
-                c_xx = fmaf(x1, x1, c_xx);
+                RS_SHIFT_OPERANDS(e)
+                c_hx = fmaf(f0, g0, c_hx);
+                c_hx = fmaf(f1, g1, c_hx);
+                c_hh = fmaf(f0, f0, c_hh);
+                c_hh = fmaf(f1, f1, c_hh);
+                c_xx = fmaf(g0, g0, c_xx);
+                c_xx = fmaf(g1, g1, c_xx);
               }
             } else if (p.dist == kDistL1) {
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
-                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
-                part += fabsf(h0 - x0);
-                part += fabsf(h1 - x1);
+                RS_SHIFT_OPERANDS(e)
+                part += fabsf(f0 - g0);
+                part += fabsf(f1 - g1);
               }
             } else {
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
-                const float h0 = __uint_as_float(r[2 * e]) + bf16lo(bw[e]);
-                const float h1 = __uint_as_float(r[2 * e + 1]) + bf16hi(bw[e]);
-                outw[e] = pack_bf16x2(x0 + h0, x1 + h1);
-                const float d0 = h0 - x0, d1 = h1 - x1;
+                RS_SHIFT_OPERANDS(e)
+                const float d0 = f0 - g0, d1 = f1 - g1;
                 part = fmaf(d0, d0, part);
                 part = fmaf(d1, d1, part);
               }
             }
+#undef RS_SHIFT_OPERANDS
           }
         }
         if (n + 1 == NCH) {

@@ -47,6 +47,8 @@ SIGNATURES = {
     "rs_select_topk": (_i, [_fp, _i, _i, _i, _i, _fp, _ip, _vp]),
     "rs_gather_rows": (_i, [_vp, _i, _i, _i, _ip, _i, _vp, _vp]),
     "rs_select_gather": (_i, [_fp, _i, _vp, _i, _i, _i, _i, _fp, _ip, _vp, _vp]),
+    "rs_block_forward_block_shift_ex": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                             _vp, _i, _i, _i, _vp, _ip, _fp, _vp]),
     "rs_mlp_forward": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_attn_core": (_i, [_vp, _i, _i, _i, _vp, _vp]),
     "rs_encoder_forward": (_i, [_vp, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp),
@@ -405,3 +407,28 @@ def rs_encoder_forward(x: torch.Tensor, layers, keep, heads: int,
     _check(lib().rs_encoder_forward(_ptr(x), B, L, C, H, int(heads), depth, ptrs, kk, _ptr(out),
                                     _stream(stream)), "rs_encoder_forward")
     return out
+
+
+def rs_block_forward_block_shift(x_in: torch.Tensor, x: torch.Tensor, W1, b1, W2, b2, gamma,
+                                 beta, keep_k: int, y_kept: Optional[torch.Tensor] = None,
+                                 kept_idx: Optional[torch.Tensor] = None,
+                                 scores: Optional[torch.Tensor] = None, stream=None,
+                                 distance="l2", cls: bool = True):
+    """rs_block_forward scored on the whole-block shift D(y, x_in): x_in [B, L, C] is the
+    block input before the attention sublayer, x = x' its output."""
+    B, L, C = x.shape
+    H = W1.shape[0]
+    dev = x.device
+    n = keep_k + (1 if cls else 0)
+    if y_kept is None:
+        y_kept = torch.empty(B, n, C, dtype=torch.bfloat16, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(B, n, dtype=torch.int32, device=dev)
+    if scores is None:
+        scores = torch.empty(B, L, dtype=torch.float32, device=dev)
+    st = lib().rs_block_forward_block_shift_ex(
+        _ptr(x_in), _ptr(x), B, L, C, H, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(gamma),
+        _ptr(beta), int(keep_k), _dist(distance), 0 if cls else RS_NO_CLS, _ptr(y_kept),
+        _ptr(kept_idx), _ptr(scores), _stream(stream))
+    _check(st, "rs_block_forward_block_shift")
+    return y_kept, kept_idx, scores

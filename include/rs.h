@@ -179,6 +179,18 @@ int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int
  * queries of a (sample, head)). 1 <= L <= RS_MAX_L, 64 heads <= RS_MAX_C. */
 int rs_attn_core(const void* qkv, int B, int L, int heads, void* out, void* stream);
 
+/* rs_block_forward_ex with the representation shift through the entire attention
+ * block (§3.3 "Operation choice" case (iii)): the score is D(x-hat, x_in), with
+ * x-hat = y = x' + MLP(LN(x')) in fp32 (before its bf16 store) and x_in [B, L, C]
+ * bf16 the block input that the attention sublayer (Eq. (5)) started from, instead
+ * of D(MLP(LN(x')), x'). Same launches (fc2's epilogue also reads x_in), outputs,
+ * distances, flags and errors as rs_block_forward_ex; x_in 16-byte aligned. */
+int rs_block_forward_block_shift_ex(const void* x_in, const void* x, int B, int L, int C, int H,
+                                    const void* W1, const void* b1, const void* W2,
+                                    const void* b2, const void* gamma, const void* beta,
+                                    int keep_k, int distance, int flags, void* y_kept,
+                                    int32_t* kept_idx, float* scores, void* stream);
+
 /*
  * Step-level entry points. rs_block_forward launches exactly these kernels in
  * this order; they are exported so that each step can be checked on its own.

@@ -6,6 +6,7 @@ may import this package.
 from .rs_oracle import (  # noqa: F401
     EPS,
     block_forward,
+    block_shift_forward,
     fc,
     finalize_scores_f32,
     gather,

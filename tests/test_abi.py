@@ -188,6 +188,25 @@ def test_encoder_and_mlp_entry_points_argument_errors():
                               None) == rs.RS_ERR_ALIGN
 
 
+def test_block_shift_entry_point_argument_errors():
+    lib = rs.lib()
+    w = FAKE
+
+    def f(x_in=FAKE, x=FAKE, B=2, L=197, C=192, H=768, k=137, dist=0, flags=0, out=FAKE,
+          idx=FAKE, sc=FAKE):
+        return lib.rs_block_forward_block_shift_ex(x_in, x, B, L, C, H, w, w, w, w, w, w, k,
+                                                   dist, flags, out, idx, sc, None)
+
+    assert f(B=0) == rs.RS_OK
+    assert f(x_in=None) == rs.RS_ERR_NULL
+    assert f(x_in=MIS) == rs.RS_ERR_ALIGN
+    assert f(x=None) == rs.RS_ERR_NULL
+    assert f(k=197) == rs.RS_ERR_KEEP_K
+    assert f(dist=7) == rs.RS_ERR_SHAPE
+    assert f(C=100) == rs.RS_ERR_SHAPE
+    assert f(sc=None) == rs.RS_ERR_NULL
+
+
 def test_library_has_no_torch_or_libcuda_link_dependency():
     out = os.popen(f"ldd {rs.LIB_PATH}").read()
     assert "libtorch" not in out and "libc10" not in out
