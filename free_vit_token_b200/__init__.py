@@ -18,6 +18,7 @@ from .rs import (  # noqa: F401
     rs_block_forward_block_shift,
     rs_encoder_forward,
     rs_fc2_residual_shift,
+    rs_debug_attn_skip_load,
     rs_debug_fc1_skip_load,
     rs_fc1_gelu_folded,
     rs_gather_rows,

@@ -313,7 +313,8 @@ int check_heads(int C, int heads) {
 }
 
 int run_attn_core(DevState& st, const void* qkv, int B, int L, int C, int heads, void* out,
-                  cudaStream_t s, bool pdl) {
+                  cudaStream_t s, bool pdl, int debug_skip_block = -1,
+                  unsigned long long timeout_ns = rs::kDefaultTimeoutNs) {
   CUtensorMap tmQ, tmKV;
   RS_TRY(make_tmap_qkv(&tmQ, qkv, B, L, C, rs::attn_q_box_rows()));
   RS_TRY(make_tmap_qkv(&tmKV, qkv, B, L, C, rs::attn_kv_box_rows()));
@@ -324,7 +325,8 @@ int run_attn_core(DevState& st, const void* qkv, int B, int L, int C, int heads,
   p.heads = heads;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = st.err;
-  p.timeout_ns = rs::kDefaultTimeoutNs;
+  p.timeout_ns = timeout_ns;
+  p.debug_skip_block = debug_skip_block;
   RS_CUDA(rs::launch_attn(tmQ, tmKV, p, s, pdl));
   return RS_OK;
 }
@@ -802,6 +804,24 @@ int rs_attn_core(const void* qkv, int B, int L, int heads, void* out, void* stre
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
   return run_attn_core(*st, qkv, B, L, C, heads, out, static_cast<cudaStream_t>(stream), false);
+}
+
+int rs_debug_attn_skip_load(const void* qkv, int B, int L, int heads, void* out, int skip_block,
+                            int timeout_us, void* stream) {
+  if (B < 0 || L < 1 || L > RS_MAX_L || heads < 1) return RS_ERR_SHAPE;
+  const int C = 64 * heads;
+  RS_TRY(check_heads(C, heads));
+  RS_TRY(check_rows(static_cast<int64_t>(B) * L, C, 3 * C));
+  if (skip_block < 0 || skip_block >= (L + 63) / 64 || timeout_us < 1 || timeout_us > 10000000)
+    return RS_ERR_SHAPE;
+  if (B == 0) return RS_OK;
+  if (!qkv || !out) return RS_ERR_NULL;
+  if (!al16(qkv) || !al16(out)) return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_attn_core(*st, qkv, B, L, C, heads, out, static_cast<cudaStream_t>(stream), false,
+                       skip_block, static_cast<unsigned long long>(timeout_us) * 1000ull);
 }
 
 int rs_attn_sublayer(const void* x, int B, int L, int C, int heads, const void* Wqkv,

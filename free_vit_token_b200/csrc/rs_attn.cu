@@ -118,9 +118,12 @@ __global__ void __launch_bounds__(kThreads, 3)
       mbar_arrive_expect_tx(q_full, kBox);
       tma_load_3d(sQ, &tmQ, q_full, head * kHd, q0, b);
       int issued = 0;
+      const bool hook = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
       for (int j = 0; j < nkb; ++j) {
         const int s = j % kKvStages;
         if (j >= kKvStages && !wait_bounded(&kv_empty[s], ((j / kKvStages) - 1) & 1, wc)) break;
+        // test hook: stop loading, so that the MMA warp's wait for this block runs out
+        if (hook && j == p.debug_skip_block) break;
         mbar_arrive_expect_tx(&k_full[s], kKvBox);
         tma_load_3d(sKs(s), &tmKV, &k_full[s], C + head * kHd, j * kKeys, b);
         mbar_arrive_expect_tx(&v_full[s], kKvBox);

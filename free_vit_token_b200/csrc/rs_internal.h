@@ -153,6 +153,8 @@ struct AttnParams {
   __nv_bfloat16* out;
   int* err;                       // device status flag
   unsigned long long timeout_ns;  // limit of one pipeline wait
+  int debug_skip_block;           // test hook: CTA (0, 0, 0) withholds this key block's
+                                  // loads and every later one (-1: off)
 };
 size_t attn_smem_bytes();
 int attn_q_box_rows();

@@ -51,6 +51,7 @@ SIGNATURES = {
                                              _vp, _i, _i, _i, _vp, _ip, _fp, _vp]),
     "rs_mlp_forward": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_attn_core": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "rs_debug_attn_skip_load": (_i, [_vp, _i, _i, _i, _vp, _i, _i, _vp]),
     "rs_encoder_forward": (_i, [_vp, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp),
                                 ctypes.POINTER(_i), _vp, _vp]),
     "rs_attn_sublayer": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -432,3 +433,13 @@ def rs_block_forward_block_shift(x_in: torch.Tensor, x: torch.Tensor, W1, b1, W2
         _ptr(kept_idx), _ptr(scores), _stream(stream))
     _check(st, "rs_block_forward_block_shift")
     return y_kept, kept_idx, scores
+
+
+def rs_debug_attn_skip_load(qkv: torch.Tensor, heads: int, out: torch.Tensor, skip_block: int,
+                            timeout_us: int, stream=None) -> None:
+    """Test hook: the attention core with one CTA's key-block loads withheld from
+    `skip_block` on; its waits time out after `timeout_us` (see rs.h)."""
+    B, L, _ = qkv.shape
+    _check(lib().rs_debug_attn_skip_load(_ptr(qkv), B, L, int(heads), _ptr(out), int(skip_block),
+                                         int(timeout_us), _stream(stream)),
+           "rs_debug_attn_skip_load")

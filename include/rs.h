@@ -173,6 +173,16 @@ int rs_attn_forward_ex(const void* x, int B, int L, int C, int heads, const void
 int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int depth,
                        const void* const* weights, const int* keep, void* out, void* stream);
 
+/* Test hook of the attention core's failure path: rs_attn_core in which the CTA of
+ * query tile 0, head 0, sample 0 withholds the loads of key block `skip_block`
+ * (blocks of 64 keys, 0 <= skip_block < ceil(L / 64)) and of every later block,
+ * with every pipeline wait limited to timeout_us microseconds (1 .. 1e7). The
+ * waits for the withheld tiles run out: the CTA records RS_ERR_DEVICE_TIMEOUT in
+ * the device flag, drains its MMAs, frees its TMEM and returns; no fault, no hang.
+ * Other arguments as for rs_attn_core. */
+int rs_debug_attn_skip_load(const void* qkv, int B, int L, int heads, void* out, int skip_block,
+                            int timeout_us, void* stream);
+
 /* The attention core alone: out [B, L, 64 heads] bf16 = per sample and head,
  * Softmax(Q K^T / 8) V from qkv [B, L, 3 * 64 heads] bf16 laid out as above (a
  * tcgen05 kernel: scores and P V in TMEM, online softmax, one CTA per 128

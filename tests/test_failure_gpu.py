@@ -38,6 +38,33 @@ def test_withheld_load_times_out_and_context_survives(M, C, H):
     assert rs.rs_get_last_device_error() == rsmod.RS_OK
 
 
+@pytest.mark.parametrize("L,skip", [(300, 2), (64, 0)])
+def test_attention_withheld_load_times_out_and_context_survives(L, skip):
+    """The attention core's waits are bounded too: one CTA's key tiles withheld from
+    block `skip` on, the MMA warp's wait runs out, the flag reads
+    RS_ERR_DEVICE_TIMEOUT, and the next ordinary call is correct."""
+    import free_vit_token_b200 as rs
+    import free_vit_token_b200.rs as rsmod
+    from oracle import attn_oracle
+    from workloads import random_qkv
+
+    dev = torch.device("cuda:0")
+    heads = 2
+    qkv = random_qkv(2, L, heads, seed=L).to(dev)
+    out = torch.zeros(2, L, 64 * heads, dtype=torch.bfloat16, device=dev)
+    assert rs.rs_get_last_device_error() == rsmod.RS_OK
+    rs.rs_debug_attn_skip_load(qkv, heads, out, skip_block=skip, timeout_us=20000)
+    assert rs.rs_get_last_device_error() == rsmod.RS_ERR_DEVICE_TIMEOUT
+    assert rs.rs_get_last_device_error() == rsmod.RS_OK
+    got = rs.rs_attn_core(qkv, heads)
+    torch.cuda.synchronize()
+    q64 = parity.f64(qkv.cpu())
+    for b in range(2):
+        parity.check_y(parity.f64(got[b].cpu()), attn_oracle.attention_core(q64[b], heads),
+                       "attention after timeout")
+    assert rs.rs_get_last_device_error() == rsmod.RS_OK
+
+
 def test_hook_argument_checks():
     import free_vit_token_b200.rs as rsmod
 
@@ -47,3 +74,5 @@ def test_hook_argument_checks():
                                     None) == rsmod.RS_ERR_SHAPE
     assert L.rs_debug_fc1_skip_load(fake, 10, 384, 1536, fake, fake, fake, fake, fake, 0, 0,
                                     None) == rsmod.RS_ERR_SHAPE
+    assert L.rs_debug_attn_skip_load(fake, 1, 300, 2, fake, 5, 1000, None) == rsmod.RS_ERR_SHAPE
+    assert L.rs_debug_attn_skip_load(fake, 1, 300, 2, fake, 0, 0, None) == rsmod.RS_ERR_SHAPE
