@@ -116,3 +116,13 @@ def test_encoder_pins_catch_mutation(name, monkeypatch):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin catches {name!r}"
+
+
+def test_bench_schedule_matches_oracle():
+    """bench.py's 12-layer timing uses the same pruning schedule as the oracle's reading
+    of §4.2 (written separately there, since bench.py's timed path does not use the
+    oracle)."""
+    import bench
+    assert bench.deit_keep_schedule(197) == encoder_oracle.deit_schedule()
+    for L in (50, 101, 577):
+        assert bench.deit_keep_schedule(L) == encoder_oracle.deit_schedule(L=L)
