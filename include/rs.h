@@ -1,6 +1,6 @@
 /*
  * rs.h -- C ABI of librs.so: the pruned-MLP block of Representation Shift on
- * NVIDIA B200 (sm_100a).
+ * NVIDIA B200 (sm_100a), and the attention sublayer and encoder layers around it.
  *
  * Method: "Representation Shift: Unifying Token Compression with
  * FlashAttention" (arXiv 2508.00367v1, ICCV 2025).
@@ -9,6 +9,9 @@
  *     D = L2 (§3.3 "Distance metrics" (i)):   s = || MLP(LN(x')) - x' ||_2
  *   - Pruning, §3.1 / §3.2: drop the lowest-s tokens, keep x-tilde in
  *     R^{(N-r) x C} for the attention layer that follows.
+ *   - Attention sublayer, §3.1 Eq. (1) and §3.3 Eq. (5): x' = SA(LN(x)) + x
+ *     (rs_attn_*), and layers of both with pruning between them
+ *     (rs_encoder_forward; the §4.2 DeiT schedule is one choice of keep[]).
  *
  * Conventions shared by every entry point:
  *   - Every tensor argument is a DEVICE pointer owned by the caller, contiguous,
@@ -29,10 +32,14 @@
  *   - Shape limits: 1 <= L <= RS_MAX_L; C and H multiples of 64 with
  *     64 <= C <= RS_MAX_C and 64 <= H <= RS_MAX_H; 0 <= keep_k <= L-1;
  *     B*L*max(C,H) < 2^31. B = 0 is an empty batch: RS_OK, nothing launched.
- *   - Library workspace: rs_block_forward and the fc steps use a per-device
- *     workspace owned by the library (cudaMalloc'd on first use, grown on
- *     demand, reused across calls). Growing it synchronises the device. Calls
- *     that share a device must be ordered on one stream (they share it).
+ *   - Library workspace: rs_block_forward, the fc steps, the attention entry
+ *     points and rs_encoder_forward use a per-device workspace owned by the
+ *     library (cudaMalloc'd on first use, grown on demand, reused across calls;
+ *     rs_encoder_forward also keeps a second buffer for its activations).
+ *     Growing either synchronises the device. Calls that share a device must be
+ *     ordered on one stream (they share the buffers). Once the buffers have
+ *     grown to a call's sizes, repeating the call allocates nothing, so it can
+ *     be captured in a CUDA graph.
  */
 #ifndef RS_H_
 #define RS_H_
