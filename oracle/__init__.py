@@ -1,4 +1,6 @@
-"""fp64 CPU oracle for the pruned-MLP block (test infrastructure, not the product).
+"""fp64 CPU oracles (test infrastructure, not the product): the pruned-MLP block
+(``rs_oracle``), the attention sublayer (``attn_oracle``) and encoder layers with
+pruning between them (``encoder_oracle``).
 
 Only tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
 may import this package.
