@@ -206,6 +206,53 @@ def oracle_rate(wl, seed: int, budget_s: float):
 
 
 # ----------------------------------------------------------------------------- main
+def time_variants(rs, wl, x, W0, out0, dev, stream, reps: int):
+    """The first stage's block with the other scores and modes the library offers,
+    against the L2 default measured the same way (mean of `reps` back-to-back calls
+    between CUDA events, inputs L2-warm): the L1 and cosine distances, no CLS token
+    (k + 1 of all L tokens ranked, the same output sizes), the whole-block shift
+    D(y, x_in) (x_in: a second [B, L, C] input), and the attention sublayer followed
+    by pruning on its own shift."""
+    if reps <= 0:
+        return None
+    from workloads import draw_attn_weights
+    k = wl.keep_k[0]
+    y_kept, kept, scores = out0
+    x_in = torch.flip(x, dims=[1]).contiguous()
+    calls = {
+        "l2": lambda: rs.rs_block_forward(x, *W0, k, y_kept, kept, scores, stream=stream),
+        "l1": lambda: rs.rs_block_forward(x, *W0, k, y_kept, kept, scores, stream=stream,
+                                          distance="l1"),
+        "cosine": lambda: rs.rs_block_forward(x, *W0, k, y_kept, kept, scores, stream=stream,
+                                              distance="cosine"),
+        "no_cls": lambda: rs.rs_block_forward(x, *W0, k + 1, y_kept, kept, scores, stream=stream,
+                                              cls=False),
+        "block_shift": lambda: rs.rs_block_forward_block_shift(x_in, x, *W0, k, y_kept, kept,
+                                                               scores, stream=stream),
+    }
+    if wl.C % 64 == 0:
+        aw = draw_attn_weights(wl.C, seed=1001)
+        Wa = [t.to(dev) for t in (aw.Wqkv, aw.bqkv, aw.Wo, aw.bo, aw.gamma, aw.beta)]
+        calls["attention_shift"] = lambda: rs.rs_attn_forward(x, *Wa, wl.C // 64, k, y_kept,
+                                                               kept, scores, stream=stream)
+    res = {"reps": reps, "timing": "mean of back-to-back calls between CUDA events, L2-warm"}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            fn()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        res[name] = {"ms": t0.elapsed_time(t1) / reps}
+    assert rs.rs_get_last_device_error() == 0
+    for name in calls:
+        res[name]["vs_l2"] = res[name]["ms"] / res["l2"]["ms"]
+    return res
+
+
 def time_attention(rs, wl, x_full, x_kept, peaks, dev, stream, reps: int):
     """The attention sublayer (x + SA(LN(x)), Eq. (5)) that the next layer runs, on
     the stage-0 input (L tokens) and on the pruned block's output (1 + k tokens):
@@ -305,6 +352,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="deit_s", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
+    ap.add_argument("--variant-reps", type=int, default=20,
+                    help="calls per score-variant timing (0: skip that measurement)")
     ap.add_argument("--encoder-reps", type=int, default=5,
                     help="calls per 12-layer encoder timing (0: skip that measurement)")
     ap.add_argument("--attn-reps", type=int, default=20,
@@ -563,6 +612,7 @@ def main():
     e2e_value = job_throughput(tokens_per_step, 1, e2e_ms, world)
     clocks.stop()
 
+    variants = time_variants(rs, wl, x, W[0], outs[0], dev, stream, args.variant_reps)
     attn = time_attention(rs, wl, x, outs[0][0], peaks, dev, stream, args.attn_reps)
     sched = time_encoder_schedule(rs, wl, x, dev, stream, args.encoder_reps)
 
@@ -608,6 +658,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (own streams)"},
+        "score_variants": variants,
         "attention_next_layer": attn,
         "encoder_schedule": sched,
         "gpu_launches": kernels_per_step(wl) * args.steps,
