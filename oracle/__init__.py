@@ -10,7 +10,6 @@ from .rs_oracle import (  # noqa: F401
     block_forward,
     block_shift_forward,
     fc,
-    finalize_scores_f32,
     gather,
     gelu,
     layer_norm,

@@ -157,38 +157,3 @@ def block_shift_forward(x_in, x, W1, b1, W2, b2, gamma, beta, keep_k: int, eps: 
     kept = np.stack([select_topk(s[b], keep_k, cls) for b in range(B)])
     y_kept = np.stack([gather(y[b], kept[b]) for b in range(B)])
     return y_kept, kept, s, y
-
-
-def finalize_scores_f32(partials: np.ndarray, B: int, L: int, metric: str = "l2") -> np.ndarray:
-    """Scores from fp32 per-row partial sums, in fp32 (correctly rounded operations).
-
-    l2:     partials are sums of (h - x)^2 over column groups; s = sqrt(sum_j P[r, j]).
-    l1:     partials are sums of |h - x|; s = sum_j P[r, j].
-    cosine: partials are triples (sum h.x, sum h.h, sum x.x) per column group;
-            s = max(0, 1 - HX / max(sqrt(HH) * sqrt(XX), COS_EPS)) with HX, HH, XX the
-            group sums. Floored at 0 so that the fp32 bits order like the values.
-    Partials are added left to right (group order). Used where an fp32 score decides
-    the integer kept set, so that both sides rank the same fp32 keys.
-    """
-    f32 = np.float32
-    p = np.asarray(partials, dtype=f32).reshape(B * L, -1)
-
-    def rsum(cols):
-        acc = np.zeros(B * L, dtype=f32)
-        for j in cols:
-            acc = (acc + p[:, j]).astype(f32)
-        return acc
-
-    if metric == "l2":
-        return np.sqrt(rsum(range(p.shape[1]))).astype(f32).reshape(B, L)
-    if metric == "l1":
-        return rsum(range(p.shape[1])).reshape(B, L)
-    if metric == "cosine":
-        if p.shape[1] % 3:
-            raise ValueError("cosine partials come in triples")
-        n = p.shape[1]
-        hx, hh, xx = rsum(range(0, n, 3)), rsum(range(1, n, 3)), rsum(range(2, n, 3))
-        den = np.maximum((np.sqrt(hh) * np.sqrt(xx)).astype(f32), f32(COS_EPS))
-        s = (f32(1.0) - (hx / den).astype(f32)).astype(f32)
-        return np.maximum(s, f32(0.0)).reshape(B, L)
-    raise ValueError(f"unknown metric {metric!r}")

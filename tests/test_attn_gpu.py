@@ -6,10 +6,13 @@ Tolerances are the MLP block's (tests/parity.py): the attention output and x' ar
 held to max|d| / max|ref| <= 2e-2 and |d| <= 2e-2 max(1, |ref|) elementwise; the
 error sources are the bf16 QKV projection, the bf16 P of the P V product, the
 SFU exp2 (relative error ~2^-22), fp32 accumulation and the bf16 stores."""
+import numpy as np
 import pytest
 import torch
 
+import kernel_model
 import parity
+from attn_cases import CONDITIONED, ILL_CONDITIONED, attn_case, case_id, w64
 from oracle import attn_oracle
 from workloads import draw_attn_weights, random_block, random_qkv
 
@@ -21,11 +24,6 @@ dev = torch.device("cuda:0")
 def _rs():
     import free_vit_token_b200 as rs  # deferred: collection must not need a GPU
     return rs
-
-
-def _w64(w):
-    return dict(Wqkv=parity.f64(w.Wqkv), bqkv=parity.f64(w.bqkv), Wo=parity.f64(w.Wo),
-                bo=parity.f64(w.bo), gamma=parity.f64(w.gamma), beta=parity.f64(w.beta))
 
 
 def _wdev(w):
@@ -72,32 +70,45 @@ def test_attn_core_empty_batch():
     assert out.shape == (0, 7, 128)
 
 
-@pytest.mark.parametrize("B,L,C,std,x_scale", [(2, 197, 384, 0.02, 1.0), (2, 138, 384, 0.05, 1.0),
-                                               (1, 300, 128, 0.05, 1.0), (3, 65, 768, 0.05, 1.0),
-                                               (1, 119, 1024, 0.02, 1.0),
-                                               (2, 197, 384, 0.05, 0.02), (1, 260, 768, 0.03, 0.02)])
-def test_attn_sublayer(B, L, C, std, x_scale):
+@pytest.mark.parametrize("case", CONDITIONED, ids=case_id)
+def test_attn_sublayer(case):
     """x' = x + SA(LN(x)): LN + QKV projection (folded-LN GEMM, no activation),
-    attention core, output projection with the residual, against the fp64 oracle.
-    With x_scale 0.02 the residual is small next to SA(LN(x)) (LN removes the
-    scale), so x' is checked mostly on the attention's own output.
-
-    The weights keep the logits' spread at about 2 or less (std 0.05 up to C = 768,
-    0.02 at C = 1024). With peaked rows (spread ~10) the sublayer is ill-conditioned
-    in its bf16 QKV projection: one bf16 ulp of q or k (relative 2^-9, the rounding
-    the projection's storage and the LN fold into bf16 weights both make) moves a
-    logit of size ~10 by ~0.02 and a softmax weight by ~2%, whatever the kernels
-    do. The attention core is checked in that regime on given bf16 Q, K, V
-    (test_attn_core, scale 3: logits of spread ~9)."""
+    attention core, output projection with the residual, against the fp64 oracle
+    and against the CPU model of the kernels' bf16 rounding points. With x scaled
+    by 0.02 the residual is small next to SA(LN(x)) (LN removes the scale), so x'
+    is checked mostly on the attention's own output."""
     rs = _rs()
-    heads = C // 64
-    inp = random_block(B, L, C, 64, seed=B * L + C, fg_rows=L // 4)
-    x = (inp.x.float() * x_scale).to(torch.bfloat16)
-    w = draw_attn_weights(C, seed=C + L, std=std)
-    got = rs.rs_attn_sublayer(x.to(dev), *_wdev(w), heads)
+    x, w = attn_case(*case)
+    heads = x.shape[2] // 64
+    got = parity.f64(rs.rs_attn_sublayer(x.to(dev), *_wdev(w), heads))
     torch.cuda.synchronize()
-    ref, _ = attn_oracle.attn_forward(parity.f64(x), heads=heads, **_w64(w))
-    parity.check_y(parity.f64(got), ref, "x'")
+    x64 = parity.f64(x)
+    ref, _ = attn_oracle.attn_forward(x64, heads=heads, **w64(w))
+    parity.check_y(got, ref, "x' vs oracle")
+    parity.check_y(got, kernel_model.attn_sublayer_bf16(x64, heads=heads, **w64(w)),
+                   "x' vs rounding model")
+    assert rs.rs_get_last_device_error() == 0
+
+
+@pytest.mark.parametrize("case", ILL_CONDITIONED, ids=case_id)
+def test_attn_sublayer_ill_conditioned(case):
+    """Inputs on which the sublayer is ill-conditioned in its bf16 operands (weights of
+    std 0.05 at C = 1024; std 0.05 with a small residual; std 0.1, nearly one-hot
+    softmax rows). The kernels' rounding points alone, modelled on the CPU, leave the
+    oracle's tolerance there (tests/test_kernel_model.py), so the kernels are held
+    to that model -- bf16(W_qkv gamma) in the LN fold, the bf16 QKV store, bf16 P
+    against the lagging row maximum, the bf16 attention output, the bf16 x' -- at the
+    same 2e-2 rule, and to the oracle on the max-abs part of the rule with 5e-2."""
+    rs = _rs()
+    x, w = attn_case(*case)
+    heads = x.shape[2] // 64
+    got = parity.f64(rs.rs_attn_sublayer(x.to(dev), *_wdev(w), heads))
+    torch.cuda.synchronize()
+    x64 = parity.f64(x)
+    parity.check_y(got, kernel_model.attn_sublayer_bf16(x64, heads=heads, **w64(w)),
+                   "x' vs rounding model")
+    ref, _ = attn_oracle.attn_forward(x64, heads=heads, **w64(w))
+    assert np.abs(got - ref).max() <= 5e-2 * np.abs(ref).max()
     assert rs.rs_get_last_device_error() == 0
 
 
@@ -116,7 +127,7 @@ def test_attn_forward_prune(metric, cls, B, L, C):
         gpu = rs.rs_attn_forward(inp.x.to(dev), *_wdev(w), heads, k, distance=metric, cls=cls)
         torch.cuda.synchronize()
         ref = attn_oracle.attn_forward(parity.f64(inp.x), heads=heads, keep_k=k, metric=metric,
-                                       cls=cls, **_w64(w))
+                                       cls=cls, **w64(w))
         parity.check_block(gpu, ref, k, cls=cls)
     assert rs.rs_get_last_device_error() == 0
 
@@ -135,6 +146,6 @@ def test_attn_sublayer_full_size(name, B, L, C, samples):
     got = rs.rs_attn_sublayer(inp.x.to(dev), *_wdev(w), heads)
     torch.cuda.synchronize()
     x64 = parity.f64(inp.x[samples])
-    ref, _ = attn_oracle.attn_forward(x64, heads=heads, **_w64(w))
+    ref, _ = attn_oracle.attn_forward(x64, heads=heads, **w64(w))
     parity.check_y(parity.f64(got[samples]), ref, name)
     assert rs.rs_get_last_device_error() == 0

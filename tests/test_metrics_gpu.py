@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 import torch
 
+import kernel_model
 import oracle
 import parity
 from workloads import WORKLOADS, make_inputs, random_block, random_partials
@@ -40,7 +41,7 @@ def test_select_metrics_bitexact(metric, cls, L, ties):
     rs = _rs()
     B = 3
     parts = _partials(B, L, metric, seed=L + 11 * ties + 5 * cls, ties=ties)
-    s_ref = oracle.finalize_scores_f32(parts.numpy(), B, L, metric)
+    s_ref = kernel_model.finalize_scores_f32(parts.numpy(), B, L, metric)
     n = L - (1 if cls else 0)  # ranked tokens
     ks = sorted({0, min(1, n), n // 2, max(n - 1, 0), n})
     pd = parts.to(dev)
@@ -78,7 +79,7 @@ def test_fc2_metric_partials(metric, M, C, H):
     x64 = parity.f64(x)
     h = oracle.fc(parity.f64(a), w64["W2"], w64["b2"])
     parity.check_y(parity.f64(y), h + x64, "y")
-    s_gpu = oracle.finalize_scores_f32(parts.cpu().numpy(), 1, M, metric)[0].astype(np.float64)
+    s_gpu = kernel_model.finalize_scores_f32(parts.cpu().numpy(), 1, M, metric)[0].astype(np.float64)
     parity.check_scores(s_gpu, oracle.shift_score(h, x64, metric))
     assert rs.rs_get_last_device_error() == 0
 

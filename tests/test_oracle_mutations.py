@@ -12,8 +12,7 @@ import oracle.rs_oracle as rs_oracle
 from oracle_pins import ALL_PINS
 
 orig = {n: getattr(rs_oracle, n) for n in
-        ["layer_norm", "gelu", "fc", "mlp", "shift_score", "select_topk", "gather", "sublayer",
-         "finalize_scores_f32"]}
+        ["layer_norm", "gelu", "fc", "mlp", "shift_score", "select_topk", "gather", "sublayer"]}
 
 
 def _ln_unbiased(x, gamma, beta, eps=rs_oracle.EPS):
@@ -161,20 +160,6 @@ def _sublayer_no_residual(x, W1, b1, W2, b2, gamma, beta, eps=rs_oracle.EPS, met
     return h, h, rs_oracle.shift_score(h, x, metric)
 
 
-def _finalize_cos_no_floor(partials, B, L, metric="l2"):
-    if metric != "cosine":
-        return orig["finalize_scores_f32"](partials, B, L, metric)
-    p = np.asarray(partials, dtype=np.float32).reshape(B * L, -1)
-    hx, hh, xx = (p[:, i::3].sum(1, dtype=np.float32) for i in range(3))
-    return (1 - hx / (np.sqrt(hh) * np.sqrt(xx) + np.float32(1e-8))).reshape(B, L)
-
-
-def _finalize_l1_sqrt(partials, B, L, metric="l2"):
-    if metric != "l1":
-        return orig["finalize_scores_f32"](partials, B, L, metric)
-    return orig["finalize_scores_f32"](partials, B, L, "l2")
-
-
 def _block_shift_vs_x_prime(x_in, x, W1, b1, W2, b2, gamma, beta, keep_k, eps=rs_oracle.EPS,
                             metric="l2", cls=True):
     # compares y with x' instead of the block input: the MLP shift of case (ii) in disguise
@@ -224,8 +209,6 @@ MUTATIONS = {
     "select_unsorted_output": ("select_topk", _for_cls(_select_unsorted)),
     "no_cls_still_keeps_cls": ("select_topk", _no_cls_still_keeps_cls),
     "no_cls_never_keeps_t0": ("select_topk", _no_cls_skips_t0),
-    "finalize_cosine_not_floored": ("finalize_scores_f32", _finalize_cos_no_floor),
-    "finalize_l1_takes_sqrt": ("finalize_scores_f32", _finalize_l1_sqrt),
     "gather_off_by_one": ("gather", _gather_shift),
     "score_after_residual": ("sublayer", _sublayer_score_after_residual),
     "no_residual": ("sublayer", _sublayer_no_residual),
