@@ -13,9 +13,46 @@
 #include "rs.h"
 #include "rs_internal.h"
 
+namespace rs {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// A 2-D bf16 tensor map (layout and swizzle choice as declared in rs_internal.h).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
+              uint32_t box_inner) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return RS_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_inner == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RS_OK : RS_ERR_CUDA;
+}
+
+}  // namespace rs
+
 namespace {
 
 constexpr int kMaxDevices = 64;
+using rs::encode_fn;
+using rs::make_tmap;
 
 struct DevState {
   void* ws = nullptr;
@@ -78,56 +115,39 @@ int dev_state(DevState** out) {
   return RS_OK;
 }
 
-// Caller holds g_mu.
-int ensure_ws(DevState& st, size_t bytes) {
-  if (st.ws_bytes >= bytes) return RS_OK;
-  if (st.ws != nullptr) {
-    cudaDeviceSynchronize();
-    cudaFree(st.ws);
-    st.ws = nullptr;
-    st.ws_bytes = 0;
-  }
-  if (cudaMalloc(&st.ws, bytes) != cudaSuccess) {
+// Caller holds g_mu. Grows a cached buffer in stream order on `s`: the old one is
+// released with cudaFreeAsync and the new one taken with cudaMallocAsync, so no
+// call synchronises the device. The buffer is shared by every call on the device
+// (calls on different streams must be ordered by the caller). It cannot grow while
+// `s` is being captured into a graph: an allocation made during capture would
+// belong to the graph, so the call fails with RS_ERR_NO_MEM and the caller makes
+// one call at the largest size before capturing.
+int grow_buffer(void** buf, size_t* cur, size_t bytes, cudaStream_t s) {
+  if (*cur >= bytes) return RS_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
     cudaGetLastError();
-    st.ws = nullptr;
+    return RS_ERR_CUDA;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return RS_ERR_NO_MEM;
+  if (*buf != nullptr) {
+    if (cudaFreeAsync(*buf, s) != cudaSuccess) {
+      cudaGetLastError();
+      return RS_ERR_CUDA;
+    }
+    *buf = nullptr;
+    *cur = 0;
+  }
+  if (cudaMallocAsync(buf, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    *buf = nullptr;
     return RS_ERR_NO_MEM;
   }
-  st.ws_bytes = bytes;
+  *cur = bytes;
   return RS_OK;
 }
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// Row-major bf16 [rows, inner] viewed as tiles of {box_inner elements, box_rows
-// rows}: 64-wide boxes use the 128-byte swizzle (GEMM operands), 16-wide boxes
-// the 32-byte swizzle (epilogue output boxes). Rows past the end read as zero
-// and are not written.
-int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
-              uint32_t box_inner = 64) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return RS_ERR_CUDA;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw = box_inner == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : box_inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RS_OK : RS_ERR_CUDA;
+int ensure_ws(DevState& st, size_t bytes, cudaStream_t s) {
+  return grow_buffer(&st.ws, &st.ws_bytes, bytes, s);
 }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -342,7 +362,7 @@ int run_attn_sublayer(DevState& st, const void* x, int B, int L, int C, int head
   const int M = static_cast<int>(M64);
   const AttnWs aw = attn_ws_layout(M64, C);
   const WsLayout& w = aw.w;
-  RS_TRY(ensure_ws(st, w.total));
+  RS_TRY(ensure_ws(st, w.total, s));
   uint8_t* ws = static_cast<uint8_t*>(st.ws);
   void* qkv = ws + w.hidden;
   void* attn_o = ws + aw.o;
@@ -365,7 +385,7 @@ int run_block(DevState& st, const void* x, int B, int L, int C, int H, const voi
               const void* shift_ref = nullptr) {
   const int M = B * L;
   const WsLayout w = ws_layout(M, C, H);
-  RS_TRY(ensure_ws(st, w.total));
+  RS_TRY(ensure_ws(st, w.total, s));
   uint8_t* ws = static_cast<uint8_t*>(st.ws);
   void* hidden = ws + w.hidden;
   void* y = ws + w.y;
@@ -386,7 +406,7 @@ int run_mlp(DevState& st, const void* x, int M, int C, int H, const void* W1, co
             const void* W2, const void* b2, const void* gamma, const void* beta, void* y,
             cudaStream_t s) {
   const WsLayout w = ws_layout(M, C, H);
-  RS_TRY(ensure_ws(st, w.total));
+  RS_TRY(ensure_ws(st, w.total, s));
   uint8_t* ws = static_cast<uint8_t*>(st.ws);
   void* hidden = ws + w.hidden;
   RS_TRY(run_fc1(st, x, M, C, H, W1, b1, gamma, beta, ws, w, hidden, false, s));
@@ -395,21 +415,9 @@ int run_mlp(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   return RS_OK;
 }
 
-// Caller holds g_mu; grows the encoder's activation buffer (stream-ordered use).
-int ensure_act(DevState& st, size_t bytes) {
-  if (st.act_bytes >= bytes) return RS_OK;
-  if (st.act != nullptr) {
-    cudaDeviceSynchronize();
-    cudaFree(st.act);
-    st.act = nullptr;
-    st.act_bytes = 0;
-  }
-  if (cudaMalloc(&st.act, bytes) != cudaSuccess) {
-    cudaGetLastError();
-    return RS_ERR_NO_MEM;
-  }
-  st.act_bytes = bytes;
-  return RS_OK;
+// Caller holds g_mu; grows the encoder's activation buffer (as the workspace).
+int ensure_act(DevState& st, size_t bytes, cudaStream_t s) {
+  return grow_buffer(&st.act, &st.act_bytes, bytes, s);
 }
 
 int check_attn_args(const void* x, int B, int L, int C, int heads, const void* Wqkv,
@@ -440,7 +448,8 @@ const char* rs_status_string(int status) {
     case RS_ERR_ALIGN: return "RS_ERR_ALIGN: a pointer is not suitably aligned";
     case RS_ERR_CUDA: return "RS_ERR_CUDA: the CUDA runtime or driver reported an error";
     case RS_ERR_DEVICE_TIMEOUT: return "RS_ERR_DEVICE_TIMEOUT: a kernel pipeline wait timed out";
-    case RS_ERR_NO_MEM: return "RS_ERR_NO_MEM: workspace allocation failed";
+    case RS_ERR_NO_MEM:
+      return "RS_ERR_NO_MEM: workspace allocation failed (or growth needed during stream capture)";
     default: return "unknown rs_status";
   }
 }
@@ -487,7 +496,7 @@ static int ln_fc1_gelu(const void* x, int M, int C, int H, const void* W1, const
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
   const WsLayout w = ws_layout(M, C, H);
-  RS_TRY(ensure_ws(*st, w.fc1_total));
+  RS_TRY(ensure_ws(*st, w.fc1_total, static_cast<cudaStream_t>(stream)));
   return run_fc1(*st, x, M, C, H, W1, b1, gamma, beta, static_cast<uint8_t*>(st->ws), w, hidden,
                  staged, static_cast<cudaStream_t>(stream));
 }
@@ -591,9 +600,9 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   DevState* st = nullptr;
   RS_TRY(dev_state(&st));
   const WsLayout w = ws_layout(M, C, H);
-  RS_TRY(ensure_ws(*st, w.fc1_total));
-  uint8_t* ws = static_cast<uint8_t*>(st->ws);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RS_TRY(ensure_ws(*st, w.fc1_total, s));
+  uint8_t* ws = static_cast<uint8_t*>(st->ws);
   float* stats = reinterpret_cast<float*>(ws + w.stats);
   void* wg = ws + w.wg;
   float* colg = reinterpret_cast<float*>(ws + w.colg);
@@ -894,7 +903,7 @@ int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int
   // kept indices and scores of a pruning layer
   const size_t xb = align_up(static_cast<size_t>(B) * L * C * 2, 1024);
   const size_t ib = align_up(static_cast<size_t>(B) * L * 4, 1024);
-  RS_TRY(ensure_act(*st, 3 * xb + 2 * ib));
+  RS_TRY(ensure_act(*st, 3 * xb + 2 * ib, s));
   uint8_t* act = static_cast<uint8_t*>(st->act);
   void* xp = act;
   void* buf[2] = {act + xb, act + 2 * xb};
@@ -904,7 +913,7 @@ int rs_encoder_forward(const void* x, int B, int L, int C, int H, int heads, int
   {
     const int64_t M = static_cast<int64_t>(B) * L;
     const size_t a = attn_ws_layout(M, C).w.total, m = ws_layout(M, C, H).total;
-    RS_TRY(ensure_ws(*st, a > m ? a : m));
+    RS_TRY(ensure_ws(*st, a > m ? a : m, s));
   }
   const void* cur = x;
   Lc = L;
@@ -936,7 +945,9 @@ int rs_get_last_device_error(void* stream) {
   int v = 0;
   RS_CUDA(cudaMemcpy(&v, st->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (v != 0) RS_CUDA(cudaMemset(st->err, 0, sizeof(int)));
-  return v;
+  // rs_ln_fc1_gelu_noalloc records its status in its own static scratch
+  const int na = rs::noalloc_take_error();
+  return v != 0 ? v : na;
 }
 
 void rs_release_workspace(void) {
@@ -948,8 +959,10 @@ void rs_release_workspace(void) {
     if (st.ws == nullptr && st.act == nullptr) continue;
     if (cudaSetDevice(d) == cudaSuccess) {
       cudaDeviceSynchronize();
-      if (st.ws) cudaFree(st.ws);
-      if (st.act) cudaFree(st.act);
+      if (st.ws) cudaFreeAsync(st.ws, 0);
+      if (st.act) cudaFreeAsync(st.act, 0);
+      cudaDeviceSynchronize();
+      cudaGetLastError();
     }
     st.ws = nullptr;
     st.ws_bytes = 0;

@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -93,6 +94,19 @@ struct MlpParams {
 };
 
 size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);
+
+// The driver's cuTensorMapEncodeTiled (resolved once through the runtime), or null.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+// Row-major bf16 [rows, inner] viewed as tiles of {box_inner elements, box_rows
+// rows}: 64-wide boxes use the 128-byte swizzle (GEMM operands), 16-wide boxes
+// the 32-byte swizzle (epilogue output boxes). Rows past the end read as zero
+// and are not written. Returns RS_OK or RS_ERR_CUDA.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
+              uint32_t box_inner = 64);
+// rs_ln_fc1_gelu_noalloc's status slot on the current device: returns it (RS_OK or
+// RS_ERR_DEVICE_TIMEOUT) and clears it, RS_OK when that entry point never ran on
+// this device, RS_ERR_CUDA when the read fails. The caller has synchronised.
+int noalloc_take_error();
 
 // CTA pairs (tcgen05 cta_group::2, 256-row tiles with B split between the two
 // CTAs) for long reductions (K >= 1024: fc2, and fc1 at C >= 1024), where the

@@ -1,16 +1,16 @@
 // rs_noalloc.cu -- rs_ln_fc1_gelu_noalloc: the LayerNorm + fc1 + GELU step of
-// rs_ln_fc1_gelu for callers that cannot allocate device memory at call time
-// (for example code that runs while a CUDA stream is being captured into a
-// graph, where cudaMalloc is not allowed, or a host framework that owns every
-// byte of device memory through its own pool). Its scratch -- the per-row LN
-// statistics and the LN-folded fc1 weights -- lives in one file-scope static
-// device array instead of the library workspace. Every GPU that loads the
-// library holds that array (kScratchBytes, about 8.6 MiB) until the process exits.
+// rs_ln_fc1_gelu for callers that cannot allocate device memory when they call:
+// a framework that owns every byte of device memory through its own pool and
+// allows no other allocation, or latency-bound code that cannot afford a
+// cudaMalloc or cudaFree, which may synchronise the whole device. Its scratch --
+// the per-row LN statistics, the LN-folded fc1 weights and a status slot -- lives
+// in one file-scope static device array instead of the library workspace. Every
+// GPU that loads the library holds that array (kScratchBytes, about 8.6 MiB)
+// until the process exits.
 #include <cstdint>
 #include <mutex>
 
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "rs.h"
@@ -54,35 +54,34 @@ int setup(int dev) {
   return RS_OK;
 }
 
-int encode_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
-               uint32_t box_inner) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return RS_ERR_CUDA;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw = box_inner == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : box_inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
-             ? RS_OK
-             : RS_ERR_CUDA;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+namespace rs {
+
+int noalloc_take_error() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RS_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    scratch = g_scratch_ptr[dev];
+  }
+  if (scratch == nullptr) return RS_OK;  // never called on this device: nothing recorded
+  int v = 0;
+  if (cudaMemcpy(&v, scratch + kOffErr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return RS_ERR_CUDA;
+  }
+  if (v != 0 && cudaMemset(scratch + kOffErr, 0, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return RS_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // namespace rs
 
 extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const void* W1,
                                       const void* b1, const void* gamma, const void* beta,
@@ -119,15 +118,17 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
     return RS_ERR_CUDA;
   const int bn = rs::fc1_block_n(H);
   CUtensorMap tmX, tmW, tmHid;
-  if (encode_map(&tmX, x, C, M, 128, 64) != RS_OK || encode_map(&tmW, wg, C, H, bn, 64) != RS_OK ||
-      encode_map(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols) != RS_OK)
+  // single-CTA tiles: the B box holds all bn rows (rs::gemm_b_box_rows(bn, false))
+  if (rs::make_tmap(&tmX, x, C, M, 128) != RS_OK ||
+      rs::make_tmap(&tmW, wg, C, H, rs::gemm_b_box_rows(bn, false)) != RS_OK ||
+      rs::make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols) != RS_OK)
     return RS_ERR_CUDA;
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
   p.K = C;
   p.n_blocks = H / bn;
-  p.num_tiles = ((M + 127) / 128) * p.n_blocks;
+  p.num_tiles = rs::gemm_num_tiles(M, p.n_blocks, /*pair=*/false);
   p.stats = reinterpret_cast<const float2*>(stats);
   p.colG = colg;
   p.colC = colc;
@@ -135,7 +136,6 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
   p.err = err;
   p.timeout_ns = rs::kDefaultTimeoutNs;
   p.debug_skip_kb = -1;
-  // single-CTA tiles: p.num_tiles and tmW's box above are the 128-row forms
   if (rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, /*pair=*/false, num_sms, st) != cudaSuccess) {
     cudaGetLastError();
     return RS_ERR_CUDA;

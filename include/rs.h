@@ -34,12 +34,18 @@
  *     B*L*max(C,H) < 2^31. B = 0 is an empty batch: RS_OK, nothing launched.
  *   - Library workspace: rs_block_forward, the fc steps, the attention entry
  *     points and rs_encoder_forward use a per-device workspace owned by the
- *     library (cudaMalloc'd on first use, grown on demand, reused across calls;
- *     rs_encoder_forward also keeps a second buffer for its activations).
- *     Growing either synchronises the device. Calls that share a device must be
- *     ordered on one stream (they share the buffers). Once the buffers have
+ *     library (grown on demand, reused across calls; rs_encoder_forward also
+ *     keeps a second buffer for its activations). Growth is stream-ordered on
+ *     the call's stream (cudaFreeAsync of the old buffer, cudaMallocAsync of the
+ *     new one from the device's default memory pool) and synchronises nothing.
+ *     Calls that share a device must be ordered on one stream, or by the
+ *     caller's events (they share the buffers, and a buffer released by growth
+ *     on one stream may still be in use by work queued on another). A call on a
+ *     stream that is being captured into a CUDA graph cannot grow a buffer: it
+ *     returns RS_ERR_NO_MEM before launching anything. Once the buffers have
  *     grown to a call's sizes, repeating the call allocates nothing, so it can
- *     be captured in a CUDA graph.
+ *     be captured. The first call on a device also allocates, once, the
+ *     device's status flag (cudaMalloc + cudaMemset): make it before capturing.
  */
 #ifndef RS_H_
 #define RS_H_
@@ -79,7 +85,8 @@ typedef enum rs_status {
   RS_ERR_ALIGN = 4,           /* a pointer is not 16-byte (tensors) / 4-byte (int, float) aligned */
   RS_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */
   RS_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up waiting on its pipeline (device flag) */
-  RS_ERR_NO_MEM = 7           /* the workspace could not be allocated */
+  RS_ERR_NO_MEM = 7           /* the workspace could not be allocated, or would have to
+                                 grow on a stream that is being captured */
 } rs_status;
 
 /*
@@ -304,25 +311,27 @@ int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, 
                    void* y_kept, void* stream);
 
 /* rs_ln_fc1_gelu without any allocation, for callers that cannot allocate
- * device memory when they call: code running while a stream is captured into
- * a CUDA graph (where cudaMalloc is not allowed), or a host framework that
- * hands out all device memory from its own pool. The paper has no counterpart;
- * this is a library convenience.
- *   Same arguments and result as rs_ln_fc1_gelu. Its scratch (LN statistics and
- *   folded fc1 weights) is one static device array of about 8.6 MiB that every
- *   GPU loading the library holds until exit; the call itself makes no
- *   cudaMalloc, cudaFree or other allocating call.
+ * device memory when they call: a framework that owns every byte of device
+ * memory through its own pool and allows no other allocation, or latency-bound
+ * code that cannot afford cudaMalloc or cudaFree, which may synchronise the
+ * whole device. The paper has no counterpart; this is a library convenience.
+ *   Same arguments and result as rs_ln_fc1_gelu. Its scratch (LN statistics,
+ *   folded fc1 weights, a status slot) is one static device array of about
+ *   8.6 MiB that every GPU loading the library holds until exit; the call
+ *   itself makes no cudaMalloc, cudaFree or other allocating call.
  *   Limits: M <= 65536 and H * C <= 4194304, beyond which it returns
  *   RS_ERR_SHAPE without launching (as for any other shape error).
  *   The first call on a device resolves the array's device address for that
  *   device (cudaGetSymbolAddress); make that first call before any stream
  *   capture begins.
  *   Every call on a device shares the one array and leaves its contents behind;
- *   each call writes every scratch byte it reads before reading it, so nothing
- *   must start at zero. Calls whose executions overlap on the GPU (different
- *   streams, no ordering between them) race on the array: order them.
- *   A pipeline timeout on this path is recorded in the array, not in the flag
- *   that rs_get_last_device_error reads. */
+ *   each call writes every scratch byte it reads before reading it. The status
+ *   slot starts at zero (the array is zero-initialised when the library loads)
+ *   and goes back to zero when it is read. Calls whose executions overlap on
+ *   the GPU (different streams, no ordering between them) race on the array:
+ *   order them.
+ *   A pipeline timeout on this path is recorded in the status slot, which
+ *   rs_get_last_device_error reads and clears. */
 int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const void* W1, const void* b1,
                            const void* gamma, const void* beta, void* hidden, void* stream);
 
@@ -342,8 +351,9 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
 const char* rs_status_string(int status);
 
 /* Synchronises `stream`, returns and clears the current device's flag
- * (RS_OK or RS_ERR_DEVICE_TIMEOUT), or RS_ERR_CUDA if the synchronisation
- * itself failed. */
+ * (RS_OK or RS_ERR_DEVICE_TIMEOUT) together with rs_ln_fc1_gelu_noalloc's
+ * status slot on that device (either one set gives RS_ERR_DEVICE_TIMEOUT), or
+ * RS_ERR_CUDA if the synchronisation or a read failed. */
 int rs_get_last_device_error(void* stream);
 
 /* Frees the library workspace of every device (synchronises each device that
