@@ -124,8 +124,8 @@ struct SelSmem {
   uint32_t* key;   // [roundup(L, 4)] score bits, zero padded
   int32_t* kept;   // [k + 1] kept token list
   uint32_t* warp;  // [33] block scan scratch
-  uint32_t* hist;  // [256] radix histogram
-  uint32_t* sel;   // [2] selected digit, count above it
+  uint32_t* hist;  // [2][256] radix histograms (alternate passes), zero on entry to a pass
+  uint32_t* sel;   // [2][2] per pass parity: selected digit, count above it
   uint32_t* rng;   // [2 * 32] per warp: smallest and largest patch key it loaded
 };
 
@@ -263,6 +263,7 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
     s.rng[2 * (threadIdx.x >> 5)] = kmin;
     s.rng[2 * (threadIdx.x >> 5) + 1] = kmax;
   }
+  for (int i = tid; i < 512; i += nt) s.hist[i] = 0;  // both radix histogram buffers
   __syncthreads();
 }
 
@@ -301,36 +302,34 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
     kmin = s.rng[2 * w] < kmin ? s.rng[2 * w] : kmin;
     kmax = s.rng[2 * w + 1] > kmax ? s.rng[2 * w + 1] : kmax;
   }
+  // Each pass: a histogram of the candidates' digit into buffer h, one barrier, the
+  // digit found by warp 0 while the other warps clear the other buffer for the next
+  // pass, one barrier. The top byte (sign and high exponent bits, few distinct values)
+  // aggregates lanes that share a digit into one atomic; lower digits take one
+  // shared atomic per candidate (measured faster than aggregating them as well).
+  int pass = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     if (kmin <= kmax && ((kmin ^ kmax) >> shift) == 0) {
       prefix |= kmin & (0xFFu << shift);
       mask |= 0xFFu << shift;
       continue;  // every key has this digit: none above it, `need` unchanged
     }
-    for (int i = tid; i < 256; i += nt) s.hist[i] = 0;
-    __syncthreads();
+    const int h = pass & 1;
+    uint32_t* hist = s.hist + 256 * h;
     for (int base = 0; base < L; base += 4 * nt) {
       const int t0 = base + 4 * tid;
       const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
       const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-      if (shift == 24) {
-        // top byte (sign and high exponent bits): few distinct values, so lanes with
-        // the same digit are aggregated into one atomic
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = t0 + i;
-          const bool cand = t >= first && t < L;
-          const uint32_t digit = cand ? (u[i] >> 24) : 256u;
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        const bool cand = t >= first && t < L && (u[i] & mask) == prefix;
+        const uint32_t digit = cand ? ((u[i] >> shift) & 0xFFu) : 256u;
+        if (shift == 24) {
           const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-          if (cand && lane == __ffs(peers) - 1) atomicAdd(&s.hist[digit], __popc(peers));
-        }
-      } else {
-        // lower digits are spread out: one atomic per candidate key
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = t0 + i;
-          if (t >= first && t < L && (u[i] & mask) == prefix)
-            atomicAdd(&s.hist[(u[i] >> shift) & 0xFFu], 1u);
+          if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        } else if (cand) {
+          atomicAdd(&hist[digit], 1u);
         }
       }
     }
@@ -340,7 +339,7 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        c[i] = s.hist[255 - 8 * lane - i];
+        c[i] = hist[255 - 8 * lane - i];
         sum += c[i];
       }
       uint32_t incl = sum;
@@ -354,19 +353,22 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (above + c[i] >= need) {
-            s.sel[0] = static_cast<uint32_t>(255 - 8 * lane - i);
-            s.sel[1] = above;
+            s.sel[2 * h] = static_cast<uint32_t>(255 - 8 * lane - i);
+            s.sel[2 * h + 1] = above;
             break;
           }
           above += c[i];
         }
       }
+    } else {
+      uint32_t* other = s.hist + 256 * (h ^ 1);  // last read by the previous pass's scan
+      for (int i = tid - 32; i < 256; i += nt - 32) other[i] = 0;
     }
     __syncthreads();
-    // s.sel is rewritten only after the next pass's first barrier: no barrier here
-    prefix |= s.sel[0] << shift;
+    prefix |= s.sel[2 * h] << shift;
     mask |= 0xFFu << shift;
-    need -= s.sel[1];
+    need -= s.sel[2 * h + 1];
+    ++pass;
   }
   // Ordered compaction: token t (first <= t < L) is kept when key_t > T, or key_t == T
   // and fewer than `need` equal keys precede it; its place among the kept tokens
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
                                                       float* __restrict__ scores,
                                                       int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
+  __shared__ uint32_t s_warp[33], s_hist[512], s_sel[4], s_rng[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_ga
     const uint4* __restrict__ y, int Cv, int S, float* __restrict__ scores,
     int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[256], s_sel[2], s_rng[64];
+  __shared__ uint32_t s_warp[33], s_hist[512], s_sel[4], s_rng[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x / S, j0 = blockIdx.x % S;

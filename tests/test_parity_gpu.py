@@ -91,6 +91,34 @@ def test_select_gather_equals_separate_steps(L, C, k):
     assert torch.equal(s1, s2) and torch.equal(k1, k2) and torch.equal(yk1, yk2)
 
 
+@pytest.mark.parametrize("B,L", [(1, 257), (2, 300), (3, 1098), (16, 1569), (16, 768),
+                                 (32, 1569), (5, 4100), (2, 16384), (37, 600)])
+@pytest.mark.parametrize("metric,cls", [("l2", True), ("l2", False), ("l1", True),
+                                        ("cosine", True), ("cosine", False)])
+def test_select_gather_long_sequences(B, L, metric, cls):
+    """The fused select+gather on long sequences (radix selection, several CTAs per
+    sample when samples are few): the bits of the standalone selection
+    (rs_select_topk) and of the gather of its kept rows, on every keep_k edge, with
+    and without ties and a CLS token, for each distance."""
+    rs = _rs()
+    C = 1024 if L <= 1569 else 128
+    P = 6 if metric == "cosine" else 8
+    nr = L - (1 if cls else 0)
+    g = torch.Generator().manual_seed(B * L)
+    y = torch.randn(B, L, C, generator=g).to(torch.bfloat16).to(dev)
+    for ties in (False, True):
+        parts = random_partials(B, L, P, seed=B + L + ties, ties=ties).to(dev)
+        for k in sorted({0, 1, nr // 3, nr - 1, nr}):
+            s1, k1 = rs.rs_select_topk(parts, B, L, k, distance=metric, cls=cls)
+            s2, k2, yk = rs.rs_select_gather(parts, y, k, distance=metric, cls=cls)
+            torch.cuda.synchronize()
+            assert torch.equal(s1, s2), (B, L, k, "scores")
+            assert torch.equal(k1, k2), (B, L, k, "kept_idx")
+            ref = torch.stack([y[b][k1[b].long()] for b in range(B)]) if k1.shape[1] else yk
+            assert torch.equal(yk, ref), (B, L, k, "y_kept")
+    _device_ok()
+
+
 # --------------------------------------------------------------------------- LN stats
 @pytest.mark.parametrize("C", [64, 192, 384, 768, 1024, 2048])
 def test_ln_stats(C):
