@@ -82,20 +82,25 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str):
+def ncu_traffic(kernel: str, workload: str, stages: int = 1):
     """DRAM bytes (read + write) per launch of `kernel` on `workload` from
-    profiles/traffic.json, or None when absent or taken on other kernel sources."""
+    profiles/traffic.json, averaged over the workload's stages (one entry per stage,
+    as `achieved` averages the stages' launches), or None when an entry is missing
+    or was taken on other kernel sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     want = gemm_source_hash()
+    per_stage = {}
     for e in d.get("entries", []):
         if e.get("kernel") == kernel and e.get("workload") == workload and \
                 e.get("source_hash") == want:
-            return float(e["dram_bytes_per_launch"])
-    return None
+            per_stage[int(e.get("stage", 0))] = float(e["dram_bytes_per_launch"])
+    if sorted(per_stage) != list(range(stages)):
+        return None
+    return sum(per_stage.values()) / stages
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -345,12 +350,298 @@ def time_encoder_schedule(rs, wl, x, dev, stream, reps: int):
     return res
 
 
+class Block:
+    """One workload's device inputs and outputs for rs_block_forward (every stage)."""
+
+    def __init__(self, rs, wl, seed: int, dev, stream):
+        self.rs, self.wl, self.dev, self.stream = rs, wl, dev, stream
+        self.inp = make_inputs(wl, seed=seed)
+        self.x = self.inp.x.to(dev)
+        self.W = [[t.to(dev) for t in (w.W1, w.b1, w.W2, w.b2, w.gamma, w.beta)]
+                  for w in self.inp.weights]
+        self.outs = [(torch.empty(wl.B, k + 1, wl.C, dtype=torch.bfloat16, device=dev),
+                      torch.empty(wl.B, k + 1, dtype=torch.int32, device=dev),
+                      torch.empty(wl.B, wl.stage_L(s), dtype=torch.float32, device=dev))
+                     for s, k in enumerate(wl.keep_k)]
+
+    def step(self, x0=None, last=None):
+        """One pass of the block (every stage); `last` replaces the last stage's outputs."""
+        wl = self.wl
+        xs = self.x if x0 is None else x0
+        for s, k in enumerate(wl.keep_k):
+            o = last if (last is not None and s == wl.stages - 1) else self.outs[s]
+            self.rs.rs_block_forward(xs, *self.W[s], k, *o, stream=self.stream)
+            xs = o[0]
+
+
+def time_steps(blk, steps: int, warmup: int, l2_flush, world: int, clocks=None):
+    """W warm-up steps, then `steps` steps each between CUDA events with an L2 flush
+    before it (outside the events); barrier + synchronise around the loop; the max
+    over ranks of the summed step times (ms)."""
+    for _ in range(warmup):
+        l2_flush()
+        blk.step()
+    torch.cuda.synchronize()
+    st = blk.rs.rs_get_last_device_error()
+    assert st == 0, blk.rs.status_string(st)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark_start = time.time()
+    for i in range(steps):
+        l2_flush()
+        ev[i][0].record(blk.stream)
+        blk.step()
+        ev[i][1].record(blk.stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    if clocks is not None:
+        clocks.mark_end = time.time()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, blk.dev)
+    st = blk.rs.rs_get_last_device_error()
+    assert st == 0, blk.rs.status_string(st)
+    return total_ms
+
+
+KERNELS = ("stats", "fold", "fc1", "fc2", "select_gather")
+
+
+def kernel_breakdown(blk, nrep: int, l2_flush):
+    """Each kernel of the block launched through its own step-level entry point between
+    CUDA events on the launch stream, after an L2 flush per chain: mean ms per launch,
+    per stage. Returns (per_stage {s: {kernel: ms}}, scratch buffers holding the last
+    stage-by-stage y and partials as fc2 left them)."""
+    rs, wl, dev, stream = blk.rs, blk.wl, blk.dev, blk.stream
+    M0 = wl.tokens(0)
+    np_ = rs.rs_num_partials(wl.C)
+    buf = dict(stats=torch.empty(M0, 2, dtype=torch.float32, device=dev),
+               Wg=torch.empty(wl.H, wl.C, dtype=torch.bfloat16, device=dev),
+               colG=torch.empty(wl.H, dtype=torch.float32, device=dev),
+               colC=torch.empty(wl.H, dtype=torch.float32, device=dev),
+               hid=torch.empty(M0 * wl.H, dtype=torch.bfloat16, device=dev),
+               y=[torch.empty(wl.tokens(s) * wl.C, dtype=torch.bfloat16, device=dev)
+                  for s in range(wl.stages)],
+               parts=[torch.empty(wl.tokens(s) * np_, dtype=torch.float32, device=dev)
+                      for s in range(wl.stages)])
+    recs = []
+    for _ in range(nrep):
+        l2_flush()
+        xs = blk.x
+        for s, k in enumerate(wl.keep_k):
+            L_s = wl.stage_L(s)
+            M = wl.B * L_s
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            x2 = xs.reshape(M, wl.C)
+            st2 = buf["stats"][:M]
+            h2 = buf["hid"][: M * wl.H].view(M, wl.H)
+            y2 = buf["y"][s].view(M, wl.C)
+            p2 = buf["parts"][s].view(M, np_)
+            W = blk.W[s]
+            o = blk.outs[s]
+            e[0].record(stream)
+            rs.rs_ln_stats(x2, stats=st2, stream=stream)
+            e[1].record(stream)
+            rs.rs_ln_fold(W[0], W[1], W[4], W[5], buf["Wg"], buf["colG"], buf["colC"],
+                          stream=stream)
+            e[2].record(stream)
+            rs.rs_fc1_gelu_folded(x2, st2, buf["Wg"], buf["colG"], buf["colC"], hidden=h2,
+                                  stream=stream)
+            e[3].record(stream)
+            rs.rs_fc2_residual_shift(h2, x2, W[2], W[3], y=y2, partials=p2, stream=stream)
+            e[4].record(stream)
+            rs.rs_select_gather(p2, y2.view(wl.B, L_s, wl.C), k, scores=o[2], kept_idx=o[1],
+                                y_kept=o[0], stream=stream)
+            e[5].record(stream)
+            recs.append((s, e))
+            xs = o[0]
+    torch.cuda.synchronize()
+    per_stage = {}
+    for s, e in recs:
+        d = per_stage.setdefault(s, {n: [] for n in KERNELS})
+        for j, n in enumerate(KERNELS):
+            d[n].append(e[j].elapsed_time(e[j + 1]))
+    return {s: {n: statistics.mean(v) for n, v in d.items()} for s, d in per_stage.items()}, buf
+
+
+def select_gather_times(blk, buf, flush_w, flush_r):
+    """Device time of one select+gather launch per stage, summed over stages (ms):
+    (L2-hot: SG_REPS launches captured in a CUDA graph and replayed, on the partials
+    and y fc2 just wrote; after an L2 flush: graph [flush, select+gather] minus graph
+    [flush], median of 7)."""
+    rs, wl, dev, stream = blk.rs, blk.wl, blk.dev, blk.stream
+    np_ = rs.rs_num_partials(wl.C)
+    hot, cold = 0.0, 0.0
+    cap_stream = torch.cuda.Stream(dev)
+    for s, k in enumerate(wl.keep_k):
+        L_s = wl.stage_L(s)
+        M = wl.B * L_s
+        y2 = buf["y"][s].view(wl.B, L_s, wl.C)
+        p2 = buf["parts"][s].view(M, np_)
+        o = blk.outs[s]
+
+        def sg(st):
+            rs.rs_select_gather(p2, y2, k, scores=o[2], kept_idx=o[1], y_kept=o[0], stream=st)
+
+        cap_stream.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            for _ in range(SG_REPS):
+                sg(cap_stream)
+        g.replay()  # replays run on the current stream (`stream`)
+        torch.cuda.synchronize()
+        reps = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            reps.append(a.elapsed_time(b) / SG_REPS)
+        hot += statistics.median(reps)
+        del g
+        gf, gfs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf, stream=cap_stream):
+            flush_w.zero_()
+            flush_r.sum()
+        with torch.cuda.graph(gfs, stream=cap_stream):
+            flush_w.zero_()
+            flush_r.sum()
+            sg(cap_stream)
+        diffs = []
+        for _ in range(7):
+            tt = []
+            for g_ in (gf, gfs):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g_.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                tt.append(a.elapsed_time(b))
+            diffs.append(tt[1] - tt[0])
+        cold += max(statistics.median(diffs), 1e-6)
+        del gf, gfs
+    st = rs.rs_get_last_device_error()
+    assert st == 0, rs.status_string(st)
+    return hot, cold
+
+
+def select_gather_bytes(rs, wl) -> int:
+    """Algorithmic bytes of select+gather over every stage: the partials and the
+    scores once, kept_idx written, the kept rows read and written."""
+    np_ = rs.rs_num_partials(wl.C)
+    n = 0
+    for s, k in enumerate(wl.keep_k):
+        M = wl.tokens(s)
+        n += M * np_ * 4 + M * 4 + wl.B * (k + 1) * 4       # select: partials in, scores + idx out
+        n += wl.B * (k + 1) * (4 + 2 * wl.C * 2)           # gather: idx in, rows in + out
+    return n
+
+
+def measure_block(blk, steps: int, warmup: int, l2_flush, flush_w, flush_r, world: int, peaks,
+                  clocks=None):
+    """The block's timed steps, its kernel breakdown, the GEMM roofline and the
+    select+gather bandwidth for one workload."""
+    rs, wl = blk.rs, blk.wl
+    tokens_per_step = sum(wl.tokens(s) for s in range(wl.stages))
+    total_ms = time_steps(blk, steps, warmup, l2_flush, world, clocks)
+    ms_per_step = total_ms / steps
+    per_stage, buf = kernel_breakdown(blk, max(10, min(steps, 200)), l2_flush)
+    kernel_ms = {n: sum(per_stage[s][n] for s in per_stage) for n in KERNELS}
+    gemm_flops = sum(2.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages))
+    fc = {}
+    for n in ("fc1", "fc2"):
+        tf = gemm_flops / (kernel_ms[n] / 1e3) / 1e12
+        fc[n] = {"ms": kernel_ms[n], "tflops": tf, "frac": tf / peaks["bf16"],
+                 "traffic": ncu_traffic(n, wl.name, wl.stages)}
+    dominant = max(("fc1", "fc2"), key=lambda n: kernel_ms[n])
+    hot, cold = select_gather_times(blk, buf, flush_w, flush_r)
+    sg_bytes = select_gather_bytes(rs, wl)
+    block_flops = 2.0 * gemm_flops
+    block_tf = block_flops / (ms_per_step / 1e3) / 1e12
+    gbs = lambda ms: sg_bytes / (ms / 1e3) / 1e9  # noqa: E731
+    return {
+        "total_ms": total_ms, "ms_per_step": ms_per_step,
+        "tokens_per_step": tokens_per_step, "dominant": dominant, "fc": fc,
+        "kernel_ms": kernel_ms,
+        "kernel_ms_per_stage": {str(s): per_stage[s] for s in per_stage} if wl.stages > 1
+        else None,
+        "block_tflops": block_tf, "block_frac_of_bf16_peak": block_tf / peaks["bf16"],
+        "block_frac_other_peaks": {"bf16_sustained": block_tf / peaks["bf16_sustained"],
+                                   "bf16_datasheet_2250": block_tf / DATASHEET_BF16_TF},
+        "select_gather": {
+            "GBps": gbs(cold), "frac_hbm": gbs(cold) / peaks["hbm"], "bytes": sg_bytes,
+            "ms": cold, "frac_of_8TBps": gbs(cold) / DATASHEET_HBM_GBS,
+            "timing": "device time per launch right after a 256 MiB L2 flush: graph [flush, "
+                      "select+gather] minus graph [flush], median of 7, summed over stages",
+            "ms_single_launch_events": kernel_ms["select_gather"],
+            "l2_hot": {"ms": hot, "GBps": gbs(hot), "frac_hbm": gbs(hot) / peaks["hbm"],
+                       "timing": f"device time per launch, {SG_REPS} launches replayed from a "
+                                 "CUDA graph, inputs as fc2 left them (L2-resident)"}},
+    }
+
+
+def time_e2e(blk, steps: int, l2_flush, world: int):
+    """End to end through the public call with host buffers: every step copies its input
+    x' from pinned host memory and its outputs (y_kept, kept_idx, scores) back to pinned
+    host memory. Steps are pipelined as a serving loop would run them: the H2D copy of
+    step i+1 and the D2H copy of step i-1 run on their own streams while step i computes
+    (two device buffers for the input and for the outputs). Returns (ms per step, H2D
+    bytes, D2H bytes)."""
+    dev, stream = blk.dev, blk.stream
+    x_h = blk.inp.x.pin_memory()
+    h2d = x_h.numel() * x_h.element_size()
+    outs_h = tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in blk.outs[-1])
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+    x_d = [torch.empty_like(blk.x) for _ in range(2)]
+    outs_d = [tuple(torch.empty_like(o) for o in blk.outs[-1]) for _ in range(2)]
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    h2d_done, comp_done, d2h_done = [], [], []
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    s_h2d.wait_stream(stream)
+    s_d2h.wait_stream(stream)
+    for i in range(steps):
+        j = i & 1
+        if i >= 2:
+            s_h2d.wait_event(comp_done[i - 2])  # step i-2 has read x_d[j]
+        with torch.cuda.stream(s_h2d):
+            x_d[j].copy_(x_h, non_blocking=True)
+        h2d_done.append(ev())
+        h2d_done[-1].record(s_h2d)
+        stream.wait_event(h2d_done[i])
+        if i >= 2:
+            stream.wait_event(d2h_done[i - 2])  # outs_d[j] has reached the host
+        l2_flush()
+        blk.step(x_d[j], last=outs_d[j])
+        comp_done.append(ev())
+        comp_done[-1].record(stream)
+        s_d2h.wait_event(comp_done[i])
+        with torch.cuda.stream(s_d2h):
+            for oh, od in zip(outs_h, outs_d[j]):
+                oh.copy_(od, non_blocking=True)
+        d2h_done.append(ev())
+        d2h_done[-1].record(s_d2h)
+    stream.wait_event(d2h_done[-1])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(t_start.elapsed_time(t_end), world, dev) / steps, h2d, d2h
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="deit_s", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="umt_l", choices=sorted(WORKLOADS))
+    ap.add_argument("--also", default="deit_b",
+                    help="second workload measured in the same run and reported under its "
+                         "own key ('' or 'none': skip)")
     ap.add_argument("--impl", default="rs", choices=["rs", "reference"])
     ap.add_argument("--variant-reps", type=int, default=20,
                     help="calls per score-variant timing (0: skip that measurement)")
@@ -362,6 +653,7 @@ def main():
                     help="seconds of oracle work for the cpu_baseline leg (0 = skip)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
+    also = None if args.also in ("", "none", args.workload) else WORKLOADS[args.also]
     # the reference arm runs on rank 0 alone and joins no process group
     world, rank, local = dist_init("nccl") if args.impl == "rs" else env_ranks()
     tokens_per_step = sum(wl.tokens(s) for s in range(wl.stages))
@@ -401,14 +693,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    inp = make_inputs(wl, seed=rank_seed(0, rank))
-    x = inp.x.to(dev)
-    W = [[t.to(dev) for t in (w.W1, w.b1, w.W2, w.b2, w.gamma, w.beta)] for w in inp.weights]
     stream = torch.cuda.current_stream(dev)
-    outs = [(torch.empty(wl.B, k + 1, wl.C, dtype=torch.bfloat16, device=dev),
-             torch.empty(wl.B, k + 1, dtype=torch.int32, device=dev),
-             torch.empty(wl.B, wl.stage_L(s), dtype=torch.float32, device=dev))
-            for s, k in enumerate(wl.keep_k)]
+    blk = Block(rs, wl, rank_seed(0, rank), dev, stream)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -416,205 +702,37 @@ def main():
         flush_w.zero_()
         flush_r.sum()
 
-    def step(x0, last=None):
-        """One pass of the block (every stage); `last` replaces the last stage's outputs."""
-        xs = x0
-        for s, k in enumerate(wl.keep_k):
-            o = last if (last is not None and s == wl.stages - 1) else outs[s]
-            rs.rs_block_forward(xs, *W[s], k, *o, stream=stream)
-            xs = o[0]
-
     clocks = ClockSampler(local)
     clocks.start()
-    for _ in range(args.warmup):
-        l2_flush()
-        step(x)
-    torch.cuda.synchronize()
-    assert rs.rs_get_last_device_error() == 0
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.mark_start = time.time()
-    for i in range(args.steps):
-        l2_flush()
-        ev[i][0].record(stream)
-        step(x)
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks.mark_end = time.time()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), world, dev)
-    status = rs.rs_get_last_device_error()
-    assert status == 0, rs.status_string(status)
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(tokens_per_step, args.steps, total_ms, world)
-
-    # ---- per-kernel breakdown (the same kernels, one step-level entry point each)
-    names = ("stats", "fold", "fc1", "fc2", "select_gather")
-    M0 = wl.tokens(0)
-    np_ = rs.rs_num_partials(wl.C)
-    stats = torch.empty(M0, 2, dtype=torch.float32, device=dev)
-    Wg = torch.empty(wl.H, wl.C, dtype=torch.bfloat16, device=dev)
-    colG = torch.empty(wl.H, dtype=torch.float32, device=dev)
-    colC = torch.empty(wl.H, dtype=torch.float32, device=dev)
-    hid = torch.empty(M0 * wl.H, dtype=torch.bfloat16, device=dev)
-    ybuf = torch.empty(M0 * wl.C, dtype=torch.bfloat16, device=dev)
-    pbuf = torch.empty(M0 * np_, dtype=torch.float32, device=dev)
-    nrep = max(10, min(args.steps, 200))
-    recs = []
-    for i in range(nrep):
-        l2_flush()
-        xs = x
-        for s, k in enumerate(wl.keep_k):
-            L_s = wl.stage_L(s)
-            M = wl.B * L_s
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-            x2 = xs.reshape(M, wl.C)
-            st2 = stats[:M]
-            h2 = hid[: M * wl.H].view(M, wl.H)
-            y2 = ybuf[: M * wl.C].view(M, wl.C)
-            p2 = pbuf[: M * np_].view(M, np_)
-            e[0].record(stream)
-            rs.rs_ln_stats(x2, stats=st2, stream=stream)
-            e[1].record(stream)
-            rs.rs_ln_fold(W[s][0], W[s][1], W[s][4], W[s][5], Wg, colG, colC, stream=stream)
-            e[2].record(stream)
-            rs.rs_fc1_gelu_folded(x2, st2, Wg, colG, colC, hidden=h2, stream=stream)
-            e[3].record(stream)
-            rs.rs_fc2_residual_shift(h2, x2, W[s][2], W[s][3], y=y2, partials=p2, stream=stream)
-            e[4].record(stream)
-            rs.rs_select_gather(p2, y2.view(wl.B, L_s, wl.C), k, scores=outs[s][2],
-                                kept_idx=outs[s][1], y_kept=outs[s][0], stream=stream)
-            e[5].record(stream)
-            recs.append((s, e))
-            xs = outs[s][0]
-    torch.cuda.synchronize()
-    per_stage = {}
-    for s, e in recs:
-        d = per_stage.setdefault(s, {n: [] for n in names})
-        for j, n in enumerate(names):
-            d[n].append(e[j].elapsed_time(e[j + 1]))
-    gemm_flops = {s: 2.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages)}
-    fc_ms = {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage) for n in ("fc1", "fc2")}
-    dominant = max(fc_ms, key=fc_ms.get)
-    flops = sum(gemm_flops.values())
-    achieved_tf = flops / (fc_ms[dominant] / 1e3) / 1e12
-    sel_ms_event = sum(statistics.mean(per_stage[s]["select_gather"]) for s in per_stage)
-    # Device time of one select+gather launch: SG_REPS launches captured in a CUDA
-    # graph and replayed (launch overhead amortised). y and the partials are the
-    # ones fc2 just wrote in the breakdown above, L2-resident as in the block.
-    sel_ms = 0.0
-    sel_ms_flushed = 0.0
-    cap_stream = torch.cuda.Stream(dev)
-    for s, k in enumerate(wl.keep_k):
-        L_s = wl.stage_L(s)
-        M = wl.B * L_s
-        y2 = ybuf[: M * wl.C].view(wl.B, L_s, wl.C)
-        p2 = pbuf[: M * np_].view(M, np_)
-        cap_stream.wait_stream(stream)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap_stream):
-            for _ in range(SG_REPS):
-                rs.rs_select_gather(p2, y2, k, scores=outs[s][2], kept_idx=outs[s][1],
-                                    y_kept=outs[s][0], stream=cap_stream)
-        g.replay()  # replays run on the current stream (`stream`)
-        torch.cuda.synchronize()
-        reps = []
-        for _ in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            g.replay()
-            b.record(stream)
-            torch.cuda.synchronize()
-            reps.append(a.elapsed_time(b) / SG_REPS)
-        sel_ms += statistics.median(reps)
-        del g
-        # the same launch right after an L2 flush: graph [flush, select+gather] minus [flush]
-        gf, gfs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gf, stream=cap_stream):
-            flush_w.zero_()
-            flush_r.sum()
-        with torch.cuda.graph(gfs, stream=cap_stream):
-            flush_w.zero_()
-            flush_r.sum()
-            rs.rs_select_gather(p2, y2, k, scores=outs[s][2], kept_idx=outs[s][1],
-                                y_kept=outs[s][0], stream=cap_stream)
-        diffs = []
-        for _ in range(7):
-            tt = []
-            for g_ in (gf, gfs):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                g_.replay()
-                b.record(stream)
-                torch.cuda.synchronize()
-                tt.append(a.elapsed_time(b))
-            diffs.append(tt[1] - tt[0])
-        sel_ms_flushed += max(statistics.median(diffs), 1e-6)
-        del gf, gfs
-    sg_bytes = 0
-    for s, k in enumerate(wl.keep_k):
-        M = wl.tokens(s)
-        sg_bytes += M * np_ * 4 + M * 4 + wl.B * (k + 1) * 4       # select: partials in, scores + idx out
-        sg_bytes += wl.B * (k + 1) * (4 + 2 * wl.C * 2)           # gather: idx in, rows in + out
-    sg_gbs = sg_bytes / (sel_ms / 1e3) / 1e9
-    block_flops = sum(4.0 * wl.tokens(s) * wl.C * wl.H for s in range(wl.stages))
-
-    # ---- end to end through the public call with host buffers: every step copies its
-    # input x' from pinned host memory and its outputs (y_kept, kept_idx, scores) back to
-    # pinned host memory. Steps are pipelined as a serving loop would run them: the H2D
-    # copy of step i+1 and the D2H copy of step i-1 run on their own streams while step i
-    # computes (two device buffers for the input and for the outputs).
-    x_h = inp.x.pin_memory()
-    h2d = x_h.numel() * x_h.element_size()
-    outs_h = tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs[-1])
-    d2h = sum(o.numel() * o.element_size() for o in outs_h)
-    x_d = [torch.empty_like(x) for _ in range(2)]
-    outs_d = [tuple(torch.empty_like(o) for o in outs[-1]) for _ in range(2)]
-    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    m = measure_block(blk, args.steps, args.warmup, l2_flush, flush_w, flush_r, world, peaks,
+                      clocks)
+    ms_per_step = m["ms_per_step"]
+    value = job_throughput(tokens_per_step, args.steps, m["total_ms"], world)
     n_e2e = max(5, min(args.steps, 100))
-    ev = lambda: torch.cuda.Event()
-    h2d_done, comp_done, d2h_done = [], [], []
-    barrier(world)
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    s_h2d.wait_stream(stream)
-    s_d2h.wait_stream(stream)
-    for i in range(n_e2e):
-        j = i & 1
-        if i >= 2:
-            s_h2d.wait_event(comp_done[i - 2])  # step i-2 has read x_d[j]
-        with torch.cuda.stream(s_h2d):
-            x_d[j].copy_(x_h, non_blocking=True)
-        h2d_done.append(ev())
-        h2d_done[-1].record(s_h2d)
-        stream.wait_event(h2d_done[i])
-        if i >= 2:
-            stream.wait_event(d2h_done[i - 2])  # outs_d[j] has reached the host
-        l2_flush()
-        step(x_d[j], last=outs_d[j])
-        comp_done.append(ev())
-        comp_done[-1].record(stream)
-        s_d2h.wait_event(comp_done[i])
-        with torch.cuda.stream(s_d2h):
-            for oh, od in zip(outs_h, outs_d[j]):
-                oh.copy_(od, non_blocking=True)
-        d2h_done.append(ev())
-        d2h_done[-1].record(s_d2h)
-    stream.wait_event(d2h_done[-1])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev) / n_e2e
+    e2e_ms, h2d, d2h = time_e2e(blk, n_e2e, l2_flush, world)
     e2e_value = job_throughput(tokens_per_step, 1, e2e_ms, world)
     clocks.stop()
 
-    variants = time_variants(rs, wl, x, W[0], outs[0], dev, stream, args.variant_reps)
-    attn = time_attention(rs, wl, x, outs[0][0], peaks, dev, stream, args.attn_reps)
-    sched = time_encoder_schedule(rs, wl, x, dev, stream, args.encoder_reps)
+    second = None
+    if also is not None:
+        b2 = Block(rs, also, rank_seed(0, rank), dev, stream)
+        steps2 = max(5, min(args.steps, 50))
+        m2 = measure_block(b2, steps2, max(3, min(args.warmup, 10)), l2_flush, flush_w, flush_r,
+                           world, peaks)
+        second = {"workload": also.name, "B": also.B, "L": also.L, "C": also.C, "H": also.H,
+                  "keep_k": list(also.keep_k), "steps": steps2,
+                  "tokens_per_s": job_throughput(m2["tokens_per_step"], steps2, m2["total_ms"],
+                                                 world),
+                  "images_per_s": world * also.B / (m2["ms_per_step"] / 1e3),
+                  **{k: v for k, v in m2.items() if k not in ("total_ms", "dominant")}}
+        sched = time_encoder_schedule(rs, also, b2.x, dev, stream, args.encoder_reps)
+        if sched is not None:
+            second["encoder_schedule"] = sched
+        del b2
+
+    variants = time_variants(rs, wl, blk.x, blk.W[0], blk.outs[0], dev, stream, args.variant_reps)
+    attn = time_attention(rs, wl, blk.x, blk.outs[0][0], peaks, dev, stream, args.attn_reps)
+    sched = time_encoder_schedule(rs, wl, blk.x, dev, stream, args.encoder_reps)
 
     cpu = None
     if rank == 0 and args.cpu_budget > 0:
@@ -623,41 +741,32 @@ def main():
                "sample": f"{n} samples of {wl.name} (all stages, one sample at a time) in "
                          f"{dt:.1f} s on the host, fp64 numpy/BLAS"}
 
-    peak_tf = peaks["bf16"]
+    dom = m["dominant"]
+    fcd = m["fc"][dom]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config,
-        "roofline": {"bound": "tensor", "kernel": f"{dominant} (tcgen05 GEMM)",
-                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": achieved_tf / peak_tf,
-                     "traffic": ncu_traffic(dominant, wl.name) if wl.stages == 1 else None,
+        "roofline": {"bound": "tensor", "kernel": f"{dom} (tcgen05 GEMM)",
+                     "achieved": fcd["tflops"], "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": fcd["frac"], "traffic": fcd["traffic"],
                      "peak_source": f"{peaks['source']} bf16 burst",
-                     "kernel_ms": fc_ms[dominant]},
-        "block_tflops": block_flops / (ms_per_step / 1e3) / 1e12,
-        "block_frac_of_bf16_peak": block_flops / (ms_per_step / 1e3) / 1e12 / peak_tf,
-        "block_frac_other_peaks": {
-            "bf16_sustained": block_flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_sustained"],
-            "bf16_datasheet_2250": block_flops / (ms_per_step / 1e3) / 1e12 / DATASHEET_BF16_TF},
-        "kernel_ms": {n: sum(statistics.mean(per_stage[s][n]) for s in per_stage)
-                      for n in names},
-        "select_gather": {"GBps": sg_gbs, "frac_hbm": sg_gbs / peaks["hbm"],
-                          "bytes": sg_bytes, "ms": sel_ms,
-                          "timing": f"device time per launch, {SG_REPS} launches replayed from a "
-                                    "CUDA graph, inputs as fc2 left them (L2-resident)",
-                          "ms_single_launch_events": sel_ms_event,
-                          "frac_of_8TBps": sg_gbs / DATASHEET_HBM_GBS,
-                          "after_l2_flush": {"ms": sel_ms_flushed,
-                                             "GBps": sg_bytes / (sel_ms_flushed / 1e3) / 1e9,
-                                             "frac_hbm": sg_bytes / (sel_ms_flushed / 1e3) / 1e9
-                                             / peaks["hbm"],
-                                             "timing": "graph [256 MiB flush, select+gather] "
-                                                       "minus graph [flush], per launch"}},
+                     "kernel_ms": fcd["ms"],
+                     "per_launch": "flops and time summed over the workload's stages; "
+                                   "traffic averaged over the stages' launches"},
+        "gemm_roofline": m["fc"],
+        "block_tflops": m["block_tflops"],
+        "block_frac_of_bf16_peak": m["block_frac_of_bf16_peak"],
+        "block_frac_other_peaks": m["block_frac_other_peaks"],
+        "kernel_ms": m["kernel_ms"],
+        "kernel_ms_per_stage": m["kernel_ms_per_stage"],
+        "select_gather": m["select_gather"],
         "images_per_s": world * wl.B / (ms_per_step / 1e3),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (own streams)"},
+        "also": second,
         "score_variants": variants,
         "attention_next_layer": attn,
         "encoder_schedule": sched,
