@@ -221,7 +221,7 @@ int run_fc1(DevState& st, const void* x, int M, int C, int H, const void* W1, co
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, wB, C, H, rs::gemm_b_box_rows(bn, pair)));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::fc1_out_box_cols(H, C, staged)));
   RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, staged, pair, st.num_sms, s, /*pdl=*/true));
   return RS_OK;
 }
@@ -234,7 +234,7 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   CUtensorMap tmH, tmW, tmY;
   RS_TRY(make_tmap(&tmH, hidden, H, M, 128));
   RS_TRY(make_tmap(&tmW, W2, H, C, rs::gemm_b_box_rows(bn, pair)));
-  RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
+  RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, rs::fc2_out_box_cols(C)));
   rs::MlpParams p{};
   p.M = M;
   p.N = C;
@@ -565,7 +565,7 @@ int rs_fc1_gelu_folded(const void* x, const float* stats, const void* Wg, const 
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, Wg, C, H, rs::gemm_b_box_rows(bn, pair)));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::fc1_out_box_cols(H, C, false)));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;
@@ -614,7 +614,7 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   CUtensorMap tmX, tmW, tmHid;
   RS_TRY(make_tmap(&tmX, x, C, M, 128));
   RS_TRY(make_tmap(&tmW, wg, C, H, rs::gemm_b_box_rows(bn, pair)));
-  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols));
+  RS_TRY(make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::fc1_out_box_cols(H, C, false)));
   rs::MlpParams p{};
   p.M = M;
   p.N = H;

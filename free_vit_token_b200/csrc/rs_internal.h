@@ -18,11 +18,24 @@ constexpr int kEpiGelu = 0;              // fc1 epilogue: + b1, erf-GELU, bf16 s
 constexpr int kEpiResidShift = 1;        // fc2 epilogue: + b2, residual, shift partials
 constexpr int kEpiGeluFold = 2;          // fc1 epilogue: folded LN (mean, rstd, G, cb), erf-GELU
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;  // one pipeline wait: 4 s
-// The GEMM epilogue writes its outputs (hidden, y) through per-warp boxes of
-// 32 rows x 16 bf16 columns with the 32-byte swizzle; output tensor maps use
-// this box.
+// The GEMM epilogue reads its accumulators 16 columns at a time and writes its
+// outputs (hidden, y) through per-warp boxes of 32 rows and up to kEpiBoxMaxCols
+// bf16 columns (a 64-byte swizzled row), one TMA store per box: wider boxes move
+// the output in fewer row transfers, which the operand loads share the TMA unit
+// with. Output tensor maps use the box of out_box_cols.
 constexpr int kEpiBoxRows = 32;
-constexpr int kEpiBoxCols = 16;
+constexpr int kEpiChunkCols = 16;
+constexpr int kEpiBoxMaxCols = 32;
+// Epilogue warps of the GEMM kernels: 16 for the folded-LN fc1 with a short
+// reduction (K <= 512), whose epilogue rivals the main loop; 8 otherwise.
+__host__ __device__ constexpr int gemm_epi_warps(bool folded_fc1, int K) {
+  return folded_fc1 && K <= 512 ? 16 : 8;
+}
+// Output box width for tiles of bn columns and ew epilogue warps (each warp owns
+// bn / (ew / 4) columns of a tile).
+__host__ __device__ constexpr int out_box_cols(int bn, int ew) {
+  return bn * 4 / ew < kEpiBoxMaxCols ? bn * 4 / ew : kEpiBoxMaxCols;
+}
 // fc2 writes this many shift partials per row and 128 x BN output tile (one per
 // epilogue column group).
 constexpr int kFc2PartialsPerTile = 2;
@@ -93,7 +106,7 @@ struct MlpParams {
                                   // this block input instead of h with x' (§3.3 case (iii))
 };
 
-size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair = false);
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, int ew, bool pair = false);
 
 // The driver's cuTensorMapEncodeTiled (resolved once through the runtime), or null.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
@@ -123,6 +136,12 @@ inline int gemm_num_tiles(int M, int n_blocks, bool pair) {
 inline int gemm_b_box_rows(int bn, bool pair) { return pair ? bn / 2 : bn; }
 int fc1_block_n(int H);
 int fc2_block_n(int C);
+// Output box columns of the fc1 kernel for these sizes (staged: the staged-LN
+// kernel) and of the fc2 kernel.
+inline int fc1_out_box_cols(int H, int C, bool staged) {
+  return out_box_cols(fc1_block_n(H), staged ? 8 : gemm_epi_warps(true, C));
+}
+inline int fc2_out_box_cols(int C) { return out_box_cols(fc2_block_n(C), 8); }
 cudaError_t launch_ln_stats(const void* x, int M, int C, float* stats, int num_sms,
                             cudaStream_t stream, bool pdl = false);
 cudaError_t launch_ln_fold(const void* W1, const void* gamma, const void* beta, const void* b1,

@@ -34,12 +34,10 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;                         // one 128-byte swizzle row of bf16
 constexpr int kAStageBytes = kBM * kBK * 2;     // 16 KB
 constexpr int kEpiWarp0 = 4;
-constexpr int kMaxEpiWarps = 16;
 constexpr int kLnWarp0 = 12;  // staged-LN kernel: after its 8 epilogue warps
 constexpr int kNumLnWarps = 4;
 constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 constexpr int kCtrlBytes = 512;                 // barriers, TMEM slot, abort flag
-constexpr int kEpiBoxBytes = kEpiBoxRows * kEpiBoxCols * 2;  // one warp's output box
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kVecMaxBytes = 2 * 256 * 4;       // one tile's column vectors (fold: G and cb)
@@ -57,16 +55,19 @@ __host__ __device__ constexpr int vec_bytes(int bn, int epi) {
 __host__ __device__ constexpr int vec_stride(int bn, int epi) {
   return (vec_bytes(bn, epi) + 127) / 128 * 128;
 }
-__host__ __device__ constexpr int fixed_smem(bool ln, int epi) {
+// The epilogue's per-warp output boxes (32 rows x out_box_cols bf16 each).
+__host__ __device__ constexpr int out_bytes(int bn, int ew) {
+  return ew * kEpiBoxRows * out_box_cols(bn, ew) * 2;
+}
+__host__ __device__ constexpr int fixed_smem(int bn, bool ln, int epi, int ew) {
   // alignment slack + control block + gamma/beta (bf16, up to RS_MAX_C each) +
   // the epilogue's per-warp output boxes + two tiles' column vectors
-  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + kMaxEpiWarps * kEpiBoxBytes +
-         2 * kVecMaxBytes;
+  return 1024 + kCtrlBytes + (ln ? 2 * RS_MAX_C * 2 : 0) + out_bytes(bn, ew) + 2 * kVecMaxBytes;
 }
-__host__ __device__ constexpr int num_stages(int bn, bool ln, int epi, bool pair) {
-  return (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn, pair) > (pair ? 8 : 6)
+__host__ __device__ constexpr int num_stages(int bn, bool ln, int epi, bool pair, int ew) {
+  return (kSmemLimit - fixed_smem(bn, ln, epi, ew)) / stage_bytes(bn, pair) > (pair ? 8 : 6)
              ? (pair ? 8 : 6)
-             : (kSmemLimit - fixed_smem(ln, epi)) / stage_bytes(bn, pair);
+             : (kSmemLimit - fixed_smem(bn, ln, epi, ew)) / stage_bytes(bn, pair);
 }
 // Epilogue warps EW: 8 (two per TMEM lane quadrant) or 16 (four). 16 pays off
 // only where the epilogue's arithmetic rivals a short main loop (fc1 with
@@ -75,9 +76,9 @@ __host__ __device__ constexpr int num_threads(bool ln, int ew) {
   return (kEpiWarp0 + ew + (ln ? kNumLnWarps : 0)) * 32;
 }
 
-size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, bool pair) {
-  return 1024 + static_cast<size_t>(num_stages(bn, ln, epi, pair)) * stage_bytes(bn, pair) +
-         kMaxEpiWarps * kEpiBoxBytes + 2 * vec_stride(bn, epi) + kCtrlBytes +
+size_t mlp_smem_bytes(int bn, bool ln, int epi, int K, int ew, bool pair) {
+  return 1024 + static_cast<size_t>(num_stages(bn, ln, epi, pair, ew)) * stage_bytes(bn, pair) +
+         out_bytes(bn, ew) + 2 * vec_stride(bn, epi) + kCtrlBytes +
          (ln ? 4 * static_cast<size_t>(K) : 0);
 }
 
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
   static_assert(!(PAIR && LN_A), "the staged-LN kernel runs on single CTAs");
   constexpr int kBRows = PAIR ? BN / 2 : BN;       // rows of the B tile this CTA loads
   constexpr int kBStageBytes = kBRows * kBK * 2;
-  constexpr int STAGES = num_stages(BN, LN_A, EPI, PAIR);
+  constexpr int STAGES = num_stages(BN, LN_A, EPI, PAIR, EW);
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;      // output rows of one tile
   constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN);
   // bytes that complete one stage's full barrier (the leader's, for a pair)
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
   constexpr int kNumEpiWarps = EW;
   static_assert(EW == 8 || EW == 16, "epilogue warps");
   static_assert(!LN_A || EW == 8, "staged-LN kernel: 8 epilogue warps");
-  constexpr int kOutBytes = kMaxEpiWarps * kEpiBoxBytes;
+  constexpr int kOutBytes = out_bytes(BN, EW);
   constexpr int kVecBytes = vec_bytes(BN, EPI);
   constexpr int kVecStride = vec_stride(BN, EPI);
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
@@ -412,16 +413,21 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
     // kNumEpiWarps/4 column groups of the BN columns, in 16-column chunks: the
     // TMEM load (and for fc2 the residual row slice) of chunk n+1 is in flight
     // while chunk n is processed. The accumulator goes back to the MMA warp as
-    // soon as its last chunk is in registers. Every chunk leaves through the
-    // warp's 32 x 16 output box (32-byte swizzle: 16-byte half j of row r at
-    // j ^ ((r >> 2) & 1)) and a TMA store; rows past M are clipped by the store.
+    // soon as its last chunk is in registers. The chunks fill the warp's output
+    // box (32 rows x kBoxCols columns, 16 or 32: the 32- or 64-byte swizzle, 16-byte
+    // unit j of row r at j ^ ((r >> 2) & 1) or j ^ ((r >> 1) & 3)), which leaves by one
+    // TMA store when full; rows past M are clipped by the store.
     constexpr int kGroups = kNumEpiWarps / 4;
     constexpr int kCols = BN / kGroups;  // columns of one warp
-    constexpr int NCH = kCols / kEpiBoxCols;
-    static_assert(kCols % kEpiBoxCols == 0, "chunking");
+    constexpr int NCH = kCols / kEpiChunkCols;
+    constexpr int kBoxCols = out_box_cols(BN, EW);
+    constexpr int CPB = kBoxCols / kEpiChunkCols;  // chunks per box
+    constexpr int kBoxBytes = kEpiBoxRows * kBoxCols * 2;
+    static_assert(kCols % kBoxCols == 0 && kBoxCols % kEpiChunkCols == 0, "chunking");
+    static_assert(kBoxCols == 16 || kBoxCols == 32, "box swizzle");
     const int q = warp & 3;
     const int grp = (warp - kEpiWarp0) >> 2;
-    uint8_t* box = sOut + (warp - kEpiWarp0) * kEpiBoxBytes;
+    uint8_t* box = sOut + (warp - kEpiWarp0) * kBoxBytes;
     const uint32_t box_u32 = smem_u32(box);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -608,18 +614,26 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&vempty[acc]);
         }
-        if (lane == 0) bulk_wait_group_read0();
-        __syncwarp();
-        const uint32_t sw = (lane >> 2) & 1;
-        sts128(box_u32 + lane * 32 + ((0u ^ sw) << 4),
-               make_uint4(outw[0], outw[1], outw[2], outw[3]));
-        sts128(box_u32 + lane * 32 + ((1u ^ sw) << 4),
-               make_uint4(outw[4], outw[5], outw[6], outw[7]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && box_live) {
-          tma_store_2d(&tmOut, box, col0 + c, row0 + q * 32);
-          bulk_commit_group();
+        if (n % CPB == 0) {
+          // the box's previous store has read it before it is written again
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+        }
+        {
+          const uint32_t u0 = static_cast<uint32_t>((n % CPB) * 2);  // 16-byte units of the chunk
+          const uint32_t sw = kBoxCols == 16 ? (lane >> 2) & 1 : (lane >> 1) & 3;
+          sts128(box_u32 + lane * (kBoxCols * 2) + ((u0 ^ sw) << 4),
+                 make_uint4(outw[0], outw[1], outw[2], outw[3]));
+          sts128(box_u32 + lane * (kBoxCols * 2) + (((u0 + 1) ^ sw) << 4),
+                 make_uint4(outw[4], outw[5], outw[6], outw[7]));
+        }
+        if (n % CPB == CPB - 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && box_live) {
+            tma_store_2d(&tmOut, box, col0 + c - (CPB - 1) * kEpiChunkCols, row0 + q * 32);
+            bulk_commit_group();
+          }
         }
       }
       if constexpr (EPI == kEpiResidShift) {
@@ -735,7 +749,7 @@ static cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                const CUtensorMap& tmOut, const MlpParams& p, int num_sms,
                                cudaStream_t stream, bool pdl) {
   auto kern = mlp_gemm_kernel<BN, LN_A, EPI, EW, PAIR>;
-  const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K, PAIR);
+  const size_t smem = mlp_smem_bytes(BN, LN_A, EPI, p.K, EW, PAIR);
   const int threads = num_threads(LN_A, EW);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -795,7 +809,7 @@ cudaError_t launch_fc1(const CUtensorMap& tmX, const CUtensorMap& tmW1, const CU
       default: return launch_gemm<64, true, kEpiGelu>(tmX, tmW1, tmHid, p, num_sms, s, pdl);
     }
   }
-  if (p.K <= 512) {
+  if (gemm_epi_warps(true, p.K) == 16) {
     switch (bn) {
       case 256: return launch_fold<256, 16>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);
       case 128: return launch_fold<128, 16>(tmX, tmW1, tmHid, p, pair, num_sms, s, pdl);

@@ -121,7 +121,8 @@ extern "C" int rs_ln_fc1_gelu_noalloc(const void* x, int M, int C, int H, const 
   // single-CTA tiles: the B box holds all bn rows (rs::gemm_b_box_rows(bn, false))
   if (rs::make_tmap(&tmX, x, C, M, 128) != RS_OK ||
       rs::make_tmap(&tmW, wg, C, H, rs::gemm_b_box_rows(bn, false)) != RS_OK ||
-      rs::make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::kEpiBoxCols) != RS_OK)
+      rs::make_tmap(&tmHid, hidden, H, M, rs::kEpiBoxRows, rs::fc1_out_box_cols(H, C, false)) !=
+          RS_OK)
     return RS_ERR_CUDA;
   rs::MlpParams p{};
   p.M = M;
