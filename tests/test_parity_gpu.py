@@ -135,9 +135,11 @@ def test_ln_stats(C):
 
 # --------------------------------------------------------------------------- GELU
 def test_gelu_apply_error_bound():
-    """The epilogue's GELU against the exact z * Phi(z) (fp64 oracle): |error| <= 1.5e-6,
-    on warps whose values all lie in |z| <= 3 (the near-range polynomial) and on warps
-    holding wider values (the full-range one)."""
+    """The epilogue's GELU against the exact z * Phi(z) (fp64 oracle): |error| <= 2e-5 on
+    warps whose values all lie in |z| <= 3 (the near-range polynomial, fitted to 1.5e-5:
+    the result is stored as bf16, whose half-spacing is >= 9.8e-5 for outputs of
+    magnitude >= 0.05) and <= 1.5e-6 on warps holding wider values (the full-range
+    one)."""
     rs = _rs()
     g = torch.Generator().manual_seed(2)
     z = torch.cat([torch.linspace(-3, 3, 262144),                 # whole warps in range
@@ -148,9 +150,11 @@ def test_gelu_apply_error_bound():
     g = rs.rs_gelu_apply(z.to(dev)).cpu().double().numpy()
     ref = oracle.gelu(z.double().numpy())
     err = np.abs(g - ref)
-    assert err.max() <= 1.5e-6, err.max()
+    assert err.max() <= 2e-5, err.max()
+    near = np.arange(z.numel()) < 262144  # the first block: whole warps in |z| <= 3
+    assert err[~near][np.abs(z.numpy()[~near]) > 3.2].max() <= 1.5e-6  # full-range warps
     small = np.abs(z.numpy()) < 1e-3
-    assert np.all(err[small] <= 1e-6 * np.abs(ref[small]) + 1e-37)
+    assert np.all(err[small] <= 2e-5 * np.abs(ref[small]) + 1e-37)
 
 
 # --------------------------------------------------------------------------- fc1 / fc2
