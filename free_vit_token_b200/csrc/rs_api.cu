@@ -255,6 +255,32 @@ int run_fc2(DevState& st, const void* hidden, const void* x, int M, int C, int H
   return RS_OK;
 }
 
+// The fused MLP (rs_fused.cu) on LN statistics and folded weights already in place.
+int run_fused_step(DevState& st, const void* x, const float* stats, const void* wg,
+                   const float* colg, const float* colc, int M, int C, int H, const void* W2,
+                   const void* b2, void* y, float* partials, cudaStream_t s, bool pdl) {
+  CUtensorMap tmX, tmWg, tmW2, tmY;
+  RS_TRY(make_tmap(&tmX, x, C, M, 128));
+  RS_TRY(make_tmap(&tmWg, wg, C, H, 128));
+  RS_TRY(make_tmap(&tmW2, W2, H, C, rs::fused_w2_rows(C)));
+  RS_TRY(make_tmap(&tmY, y, C, M, rs::kEpiBoxRows, 16));
+  rs::FusedParams p{};
+  p.M = M;
+  p.C = C;
+  p.H = H;
+  p.num_m = (M + 127) / 128;
+  p.stats = reinterpret_cast<const float2*>(stats);
+  p.colG = colg;
+  p.colC = colc;
+  p.b2 = static_cast<const __nv_bfloat16*>(b2);
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.partials = partials;
+  p.err = st.err;
+  p.timeout_ns = rs::kDefaultTimeoutNs;
+  RS_CUDA(rs::launch_mlp_fused(tmX, tmWg, tmW2, tmY, p, st.num_sms, s, pdl));
+  return RS_OK;
+}
+
 // The distance (RS_DIST_*) and the flags (RS_NO_CLS) of an extended entry point.
 int check_mode(int distance, int flags) {
   if (distance != RS_DIST_L2 && distance != RS_DIST_L1 && distance != RS_DIST_COSINE)
@@ -630,6 +656,27 @@ int rs_debug_fc1_skip_load(const void* x, int M, int C, int H, const void* W1, c
   p.debug_skip_kb = skip_kblock;
   RS_CUDA(rs::launch_fc1(tmX, tmW, tmHid, p, bn, false, pair, st->num_sms, s));
   return RS_OK;
+}
+
+int rs_mlp_fused_supported(int C, int H) { return rs::fused_supported(C, H) ? 1 : 0; }
+
+int rs_mlp_fused(const void* x, const float* stats, const void* Wg, const float* colG,
+                 const float* colC, int M, int C, int H, const void* W2, const void* b2, void* y,
+                 float* partials, void* stream) {
+  RS_TRY(check_width(C));
+  RS_TRY(check_hidden(H));
+  RS_TRY(check_rows(M, C, H));
+  if (!rs::fused_supported(C, H)) return RS_ERR_SHAPE;
+  if (M == 0) return RS_OK;
+  if (!x || !stats || !Wg || !colG || !colC || !W2 || !b2 || !y || !partials) return RS_ERR_NULL;
+  if (!al16(x) || !al8(stats) || !al16(Wg) || !al16(colG) || !al16(colC) || !al16(W2) ||
+      !al16(b2) || !al16(y) || !al4(partials))
+    return RS_ERR_ALIGN;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevState* st = nullptr;
+  RS_TRY(dev_state(&st));
+  return run_fused_step(*st, x, stats, Wg, colG, colC, M, C, H, W2, b2, y, partials,
+                        static_cast<cudaStream_t>(stream), false);
 }
 
 int rs_gelu_apply(const float* z, float* out, int n, void* stream) {

@@ -161,6 +161,32 @@ cudaError_t launch_gelu(const float* z, float* out, int n, cudaStream_t stream);
 cudaError_t launch_fc2(const CUtensorMap& tmHid, const CUtensorMap& tmW2, const CUtensorMap& tmY,
                        const MlpParams& p, int bn, bool pair, int num_sms, cudaStream_t s,
                        bool pdl = false);
+// The fused MLP kernel (rs_fused.cu): fc1, GELU, fc2, residual and shift partials
+// in one kernel, for narrow blocks.
+constexpr int kFusedMaxC = 384;    // fc2's fp32 accumulator (C columns) + 128 in TMEM
+constexpr int kFusedPartials = 4;  // shift partials per row (one per column quarter)
+inline bool fused_supported(int C, int H) {
+  return C >= 64 && C % 64 == 0 && C <= kFusedMaxC && H >= 128 && H % 128 == 0;
+}
+struct FusedParams {
+  int M, C, H, num_m;             // rows, width, hidden width, ceil(M / 128)
+  const float2* stats;            // [M] (mean, rstd)
+  const float* colG;              // [H] sum_c Wg[j, c]
+  const float* colC;              // [H] sum_c W1[j, c] beta[c] + b1[j]
+  const __nv_bfloat16* b2;        // [C]
+  const __nv_bfloat16* x;         // [M, C] x' (residual)
+  float* partials;                // [M, kFusedPartials]
+  int* err;                       // device status flag
+  unsigned long long timeout_ns;  // limit of one pipeline wait
+};
+// Rows of W2 per TMA box and fc2 MMA (N): 128 when C is a multiple of 128, else 64.
+int fused_w2_rows(int C);
+// tmX: x' [M, C], box 64 x 128; tmWg: Wg [H, C], box 64 x 128; tmW2: W2 [C, H], box
+// 64 x fused_w2_rows(C); tmY: y [M, C], box 16 x 32 (the 32-byte swizzle).
+cudaError_t launch_mlp_fused(const CUtensorMap& tmX, const CUtensorMap& tmWg,
+                             const CUtensorMap& tmW2, const CUtensorMap& tmY, const FusedParams& p,
+                             int num_sms, cudaStream_t stream, bool pdl = false);
+
 // Selection: `dist` says how partials make a score (kDist*), `cls` whether t = 0 is a
 // CLS token (kept first, never ranked) or ranked like the others. kept_idx holds
 // cls + keep_k entries per sample.

@@ -57,6 +57,8 @@ SIGNATURES = {
     "rs_attn_sublayer": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "rs_attn_forward_ex": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
                                 _vp, _ip, _fp, _vp]),
+    "rs_mlp_fused_supported": (_i, [_i, _i]),
+    "rs_mlp_fused": (_i, [_vp, _fp, _vp, _fp, _fp, _i, _i, _i, _vp, _vp, _vp, _fp, _vp]),
     "rs_status_string": (ctypes.c_char_p, [_i]),
     "rs_get_last_device_error": (_i, [_vp]),
     "rs_release_workspace": (None, []),
@@ -218,6 +220,31 @@ def rs_ln_fc1_gelu_noalloc(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: torch
                                       _ptr(beta), _ptr(hidden), _stream(stream))
     _check(st, "rs_ln_fc1_gelu_noalloc")
     return hidden
+
+
+RS_FUSED_PARTIALS = 4
+
+
+def rs_mlp_fused_supported(C: int, H: int) -> bool:
+    return bool(lib().rs_mlp_fused_supported(int(C), int(H)))
+
+
+def rs_mlp_fused(x2d: torch.Tensor, stats: torch.Tensor, Wg: torch.Tensor, colG: torch.Tensor,
+                 colC: torch.Tensor, W2, b2, y: Optional[torch.Tensor] = None,
+                 partials: Optional[torch.Tensor] = None, stream=None
+                 ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The fused MLP on LN statistics and folded weights: (y [M, C] bf16,
+    partials [M, RS_FUSED_PARTIALS] fp32)."""
+    M, C = x2d.shape
+    H = Wg.shape[0]
+    if y is None:
+        y = torch.empty(M, C, dtype=torch.bfloat16, device=x2d.device)
+    if partials is None:
+        partials = torch.empty(M, RS_FUSED_PARTIALS, dtype=torch.float32, device=x2d.device)
+    st = lib().rs_mlp_fused(_ptr(x2d), _ptr(stats), _ptr(Wg), _ptr(colG), _ptr(colC), M, C, H,
+                            _ptr(W2), _ptr(b2), _ptr(y), _ptr(partials), _stream(stream))
+    _check(st, "rs_mlp_fused")
+    return y, partials
 
 
 def rs_debug_fc1_skip_load(x2d: torch.Tensor, W1, b1, gamma, beta, hidden: torch.Tensor,

@@ -303,6 +303,31 @@ int rs_select_gather_ex(const float* partials, int num_partials, const void* y, 
                         int C, int keep_k, int distance, int flags, float* scores,
                         int32_t* kept_idx, void* y_kept, void* stream);
 
+/* The MLP sublayer (§3.3 Eq. (6)) with the shift partials (Eq. (4)) in one
+ * kernel, for narrow blocks: fc1 with the folded LayerNorm and GELU, fc2 with
+ * b2 and the residual, the hidden activation kept on chip (TMEM, then shared
+ * memory as fc2's A operand, one 128-column chunk at a time) and never stored.
+ * Inputs as for rs_fc1_gelu_folded (stats from rs_ln_stats; Wg, colG, colC
+ * from rs_ln_fold) plus W2 [C, H] and b2 [C] bf16:
+ *   a = bf16(GELU(rstd*(x' Wg^T - mean*G) + cb)), h = a W2^T + b2 (fp32),
+ *   y = bf16(x' + h)  [M, C] bf16 output,
+ *   partials[r, j] = sum over column quarter j (columns jC/4 .. (j+1)C/4-1) of
+ *                    (h[r,c] - x'[r,c])^2, [M, RS_FUSED_PARTIALS] fp32 output
+ *                    (4-byte aligned); summed left to right they give s_t^2
+ *                    (rs_select_topk / rs_select_gather with num_partials = 4).
+ * rs_mlp_fused_supported(C, H) is 1 when 64 <= C <= 384 (C a multiple of 64)
+ * and H is a multiple of 128, else 0; rs_mlp_fused returns RS_ERR_SHAPE outside
+ * that range. It uses no workspace. rs_block_forward does not take this path:
+ * one CTA owns a 128-row tile for the whole hidden loop, so the tensor cores
+ * wait on each chunk's GELU and a short M leaves most SMs idle; the two GEMMs
+ * measured faster on a B200 at every size tried (M = 394, C = 192, H = 768:
+ * 25 against 36 us; M = 50432, C = 384, H = 1536: 150 against 221 us). */
+#define RS_FUSED_PARTIALS 4
+int rs_mlp_fused_supported(int C, int H);
+int rs_mlp_fused(const void* x, const float* stats, const void* Wg, const float* colG,
+                 const float* colC, int M, int C, int H, const void* W2, const void* b2, void* y,
+                 float* partials, void* stream);
+
 /* Row gather, the pruned set x-tilde (§3.1):
  * y_kept[b, j, :] = y[b, kept_idx[b, j], :]. y [B, L, C] bf16; kept_idx
  * [B, 1+keep_k] int32 with entries in 0..L-1 (not checked on the device);

@@ -188,6 +188,26 @@ def test_encoder_and_mlp_entry_points_argument_errors():
                               None) == rs.RS_ERR_ALIGN
 
 
+def test_fused_mlp_entry_point_argument_errors():
+    lib = rs.lib()
+
+    def f(x=FAKE, st=FAKE, M=300, C=384, H=1536, y=FAKE, part=FAKE):
+        return lib.rs_mlp_fused(x, st, FAKE, FAKE, FAKE, M, C, H, FAKE, FAKE, y, part, None)
+
+    assert lib.rs_mlp_fused_supported(384, 1536) == 1
+    assert lib.rs_mlp_fused_supported(64, 128) == 1
+    assert lib.rs_mlp_fused_supported(448, 1792) == 0    # wider than TMEM holds with T1
+    assert lib.rs_mlp_fused_supported(384, 1600) == 0    # hidden width not in 128 chunks
+    assert f(M=0) == rs.RS_OK
+    assert f(C=448, H=1792) == rs.RS_ERR_SHAPE
+    assert f(C=100) == rs.RS_ERR_SHAPE
+    assert f(x=None) == rs.RS_ERR_NULL
+    assert f(part=None) == rs.RS_ERR_NULL
+    assert f(x=MIS) == rs.RS_ERR_ALIGN
+    assert f(st=FAKE + 4) == rs.RS_ERR_ALIGN
+    assert f(part=FAKE + 2) == rs.RS_ERR_ALIGN
+
+
 def test_block_shift_entry_point_argument_errors():
     lib = rs.lib()
     w = FAKE

@@ -238,6 +238,44 @@ def test_fc2_residual_shift(M, C, H):
     _device_ok()
 
 
+@pytest.mark.parametrize("M,C,H", [(394, 192, 768), (300, 384, 1536), (130, 384, 1536),
+                                   (77, 128, 256), (1, 64, 128), (259, 320, 640), (1000, 256, 512)])
+def test_mlp_fused(M, C, H):
+    """The fused MLP (fc1, folded LN, GELU, fc2, b2, residual and shift partials with the
+    hidden activation kept on chip) vs the oracle in fp64, and vs the two-GEMM path on
+    the same LN statistics and folded weights. Widths take both fc2 piece sizes
+    (C % 128 == 0 or not) and one to six fc1 k-blocks; M takes ragged last tiles and
+    several tiles per CTA."""
+    rs = _rs()
+    assert rs.rs_mlp_fused_supported(C, H)
+    inp = random_block(1, M, C, H, seed=M + 7 * C, fg_rows=M // 4)
+    x = inp.x.reshape(M, C)
+    w = inp.weights[0]
+    xd = x.to(dev)
+    W1, b1, W2, b2, g, be = _to_dev(w)
+    stats = rs.rs_ln_stats(xd)
+    Wg, cg, cc = rs.rs_ln_fold(W1, b1, g, be)
+    y, parts = rs.rs_mlp_fused(xd, stats, Wg, cg, cc, W2, b2)
+    torch.cuda.synchronize()
+    assert parts.shape == (M, rs.RS_FUSED_PARTIALS)
+    w64 = parity.weights64(w)
+    _, y_ref, s_ref = oracle.sublayer(parity.f64(x), w64["W1"], w64["b1"], w64["W2"],
+                                      w64["b2"], w64["gamma"], w64["beta"])
+    parity.check_y(parity.f64(y), y_ref, "y (fused)")
+    s_gpu = np.sqrt(parts.double().cpu().numpy().sum(1))
+    parity.check_scores(s_gpu, s_ref)
+    # the two-GEMM path on the same device inputs: the same y and scores up to the
+    # fp32 summation order and a bf16 rounding of y
+    hid = rs.rs_fc1_gelu_folded(xd, stats, Wg, cg, cc)
+    y2, parts2 = rs.rs_fc2_residual_shift(hid, xd, W2, b2)
+    torch.cuda.synchronize()
+    dy = (y.float() - y2.float()).abs().max().item()
+    assert dy <= 2e-2 * max(1.0, y2.float().abs().max().item()), dy
+    s2 = np.sqrt(parts2.double().cpu().numpy().sum(1))
+    assert np.allclose(s_gpu, s2, rtol=1e-4, atol=1e-6)
+    _device_ok()
+
+
 # --------------------------------------------------------------------------- whole block
 def _run_block(x, w, k):
     rs = _rs()
