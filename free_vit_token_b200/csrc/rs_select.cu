@@ -13,9 +13,12 @@
 // t) -- CLS first, never ranked; without, all L tokens are ranked.
 //   * L <= 256: every thread holds one key and counts its beaters in one sweep
 //     over shared memory; an ordered ballot compaction follows.
-//   * longer L: a 4-pass MSB-first radix select finds the k-th largest key T
-//     and how many keys equal to T are kept; the ordered compaction keeps every
-//     key > T and the lowest-index keys == T.
+//   * longer L: an MSB-first radix select finds the k-th largest key T and how
+//     many keys equal to T are kept; the ordered compaction keeps every key > T
+//     and the lowest-index keys == T. It ranks key - kmin (kmin the smallest ranked
+//     key), whose digits start at the highest set bit of kmax - kmin, so the first
+//     digit already spreads the keys over the bins, and it stops refining as soon
+//     as the bin holding the k-th key has at most 32 keys: one warp ranks those.
 // Kernels: select (one CTA per sample), gather (warps share out each sample's
 // kept rows), and select+gather fused (B x S CTAs: each CTA selects its
 // sample's rows and copies every S-th kept row, so the copy spreads over the GPU).
@@ -123,14 +126,16 @@ __device__ __forceinline__ uint32_t count_beaters(const uint32_t* s_key, int L, 
 struct SelSmem {
   uint32_t* key;   // [roundup(L, 4)] score bits, zero padded
   int32_t* kept;   // [k + 1] kept token list
-  uint32_t* warp;  // [33] block scan scratch
-  uint32_t* hist;  // [2][256] radix histograms (alternate passes), zero on entry to a pass
-  uint32_t* sel;   // [2][2] per pass parity: selected digit, count above it
+  uint32_t* warp;  // [64] block scan scratch
+  uint32_t* hist;  // [3][256] radix histograms (pass p uses p % 3), zero on entry to a pass
+  uint32_t* sel;   // [8]: [0] T and [1] need from the candidate ranking; [6] counts
+                   // the keys listed in cand (zero on entry to the selection)
   uint32_t* rng;   // [2 * 32] per warp: smallest and largest patch key it loaded
+  uint32_t* cand;  // [2 * 32]: the final bin's keys [0, 32) and their tokens [32, 64)
 };
 
 __device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, uint32_t* s_hist,
-                                         uint32_t* s_sel, uint32_t* s_rng) {
+                                         uint32_t* s_sel, uint32_t* s_rng, uint32_t* s_cand) {
   SelSmem s;
   s.key = reinterpret_cast<uint32_t*>(dyn);
   s.kept = reinterpret_cast<int32_t*>(dyn + ((L + 3) & ~3) * 4);
@@ -138,6 +143,7 @@ __device__ __forceinline__ SelSmem carve(uint8_t* dyn, int L, uint32_t* s_warp, 
   s.hist = s_hist;
   s.sel = s_sel;
   s.rng = s_rng;
+  s.cand = s_cand;
   return s;
 }
 
@@ -263,7 +269,9 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
     s.rng[2 * (threadIdx.x >> 5)] = kmin;
     s.rng[2 * (threadIdx.x >> 5) + 1] = kmax;
   }
-  for (int i = tid; i < 512; i += nt) s.hist[i] = 0;  // both radix histogram buffers
+  for (int i = tid; i < 768; i += nt) s.hist[i] = 0;  // the radix histogram buffers
+  if (tid == 0) s.sel[6] = 0;
+  if (tid < 64) s.cand[tid] = 0u;
   __syncthreads();
 }
 
@@ -293,90 +301,141 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
   // gives thread tid the four keys t = base + 4 tid .. +3 (one 16-byte load).
   const int Lpad = (L + 3) & ~3;
   const uint4* key4 = reinterpret_cast<const uint4*>(s.key);
-  uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
-  // Every ranked key lies in [kmin, kmax] (as unsigned integers), so the leading bits
-  // on which kmin and kmax agree are those of every key: such digits are taken
-  // without a histogram pass (typically the top byte: sign and high exponent bits).
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int w = 0; w < (nt >> 5); ++w) {
-    kmin = s.rng[2 * w] < kmin ? s.rng[2 * w] : kmin;
-    kmax = s.rng[2 * w + 1] > kmax ? s.rng[2 * w + 1] : kmax;
+  // Every ranked key lies in [kmin, kmax] (as unsigned integers). The select runs on
+  // v = key - kmin in [0, kmax - kmin], which orders like the keys; its first digit
+  // takes the 8 bits below the highest set bit of kmax - kmin, so it spreads the keys
+  // over at least 128 bins however the range sits against powers of two (the fp32
+  // exponent field). Every warp reduces the per-warp ranges itself.
+  const int nw = nt >> 5;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = lane; i < 2 * nw; i += 32) {
+    const uint32_t v = s.rng[i];
+    if (i & 1) hi = v > hi ? v : hi;
+    else lo = v < lo ? v : lo;
   }
-  // Each pass: a histogram of the candidates' digit into buffer h, one barrier, the
-  // digit found by warp 0 while the other warps clear the other buffer for the next
-  // pass, one barrier. The top byte (sign and high exponent bits, few distinct values)
-  // aggregates lanes that share a digit into one atomic; lower digits take one
-  // shared atomic per candidate (measured faster than aggregating them as well).
-  int pass = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    if (kmin <= kmax && ((kmin ^ kmax) >> shift) == 0) {
-      prefix |= kmin & (0xFFu << shift);
-      mask |= 0xFFu << shift;
-      continue;  // every key has this digit: none above it, `need` unchanged
-    }
-    const int h = pass & 1;
-    uint32_t* hist = s.hist + 256 * h;
-    for (int base = 0; base < L; base += 4 * nt) {
-      const int t0 = base + 4 * tid;
-      const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
-      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+  const uint32_t kmin = __reduce_min_sync(0xffffffffu, lo);
+  const uint32_t kmax = __reduce_max_sync(0xffffffffu, hi);
+  uint32_t T, need = static_cast<uint32_t>(k);  // keys == T kept, lowest index first
+  if (kmin == kmax) {
+    T = kmin;  // every ranked key is the same
+  } else {
+    int hb = 31 - __clz(kmax - kmin);  // highest bit of any v
+    uint32_t mask = hb == 31 ? 0u : ~0u << (hb + 1);
+    uint32_t prefix = 0;  // every v is zero above hb
+    // Each pass: a histogram of the candidates' digit (bits hb .. shift of v, at most
+    // 8) into buffer p % 3, one barrier, then every warp scans it for the bin holding
+    // the need-th key. Buffer p % 3 is next written in pass p + 3 and zeroed during
+    // pass p + 2, after every warp has passed the barrier of pass p + 1 and with it
+    // its own scan of pass p.
+    for (int pass = 0;; ++pass) {
+      const int shift = hb >= 7 ? hb - 7 : 0;
+      const uint32_t dmask = (2u << (hb - shift)) - 1u;
+      uint32_t* hist = s.hist + 256 * (pass % 3);
+      if (pass >= 2) {
+        uint32_t* next = s.hist + 256 * ((pass + 1) % 3);
+        for (int i = tid; i < 256; i += nt) next[i] = 0;
+      }
+      for (int base = 0; base < L; base += 4 * nt) {
+        const int t0 = base + 4 * tid;
+        const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = t0 + i;
-        const bool cand = t >= first && t < L && (u[i] & mask) == prefix;
-        const uint32_t digit = cand ? ((u[i] >> shift) & 0xFFu) : 256u;
-        if (shift == 24) {
-          const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-          if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-        } else if (cand) {
-          atomicAdd(&hist[digit], 1u);
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + i;
+          const uint32_t v = u[i] - kmin;
+          if (t >= first && t < L && (v & mask) == prefix) atomicAdd(&hist[(v >> shift) & dmask], 1u);
         }
       }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns digits 255-8l .. 248-8l (lane 0 the highest)
-      uint32_t c[8], sum = 0;
+      __syncthreads();
+      // lane l owns digits 255-8l .. 248-8l (lane 0 the highest), two 16-byte loads
+      const uint4* h4 = reinterpret_cast<const uint4*>(hist) + (62 - 2 * lane);
+      const uint4 qlo = h4[0], qhi = h4[1];
+      const uint32_t c[8] = {qhi.w, qhi.z, qhi.y, qhi.x, qlo.w, qlo.z, qlo.y, qlo.x};
+      uint32_t sum = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[255 - 8 * lane - i];
-        sum += c[i];
-      }
+      for (int i = 0; i < 8; ++i) sum += c[i];
       uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
       }
-      uint32_t above = incl - sum;
-      if (above < need && need <= incl) {
+      uint32_t above = incl - sum, digit = 0, in_bin = 0;
+      const bool here = above < need && need <= incl;
+      if (here) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (above + c[i] >= need) {
-            s.sel[2 * h] = static_cast<uint32_t>(255 - 8 * lane - i);
-            s.sel[2 * h + 1] = above;
+            digit = static_cast<uint32_t>(255 - 8 * lane - i);
+            in_bin = c[i];
             break;
           }
           above += c[i];
         }
       }
-    } else {
-      uint32_t* other = s.hist + 256 * (h ^ 1);  // last read by the previous pass's scan
-      for (int i = tid - 32; i < 256; i += nt - 32) other[i] = 0;
+      const int src = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      in_bin = __shfl_sync(0xffffffffu, in_bin, src);
+      need -= __shfl_sync(0xffffffffu, above, src);  // now 1 <= need <= in_bin
+      prefix |= digit << shift;
+      mask |= dmask << shift;
+      if (shift == 0) {
+        T = prefix + kmin;  // the whole key is known
+        break;
+      }
+      if (in_bin <= 32) {
+        // The bin's keys into s.cand in any order, one barrier; every lane of warp 0
+        // ranks one of them against all (key descending, token ascending): the
+        // need-th is the k-th ranked key overall, T its key, and the keys == T that
+        // are kept are `need` minus the bin's keys above T; one barrier.
+        for (int base = 0; base < L; base += 4 * nt) {
+          const int t0 = base + 4 * tid;
+          const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
+          const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = t0 + i;
+            if (t >= first && t < L && ((u[i] - kmin) & mask) == prefix) {
+              const uint32_t slot = atomicAdd(&s.sel[6], 1u);
+              s.cand[slot] = u[i];
+              s.cand[32 + slot] = static_cast<uint32_t>(t);
+            }
+          }
+        }
+        __syncthreads();
+        if (warp == 0) {
+          // lane l holds candidate l; the others come by shuffle, one per step
+          const bool mine = static_cast<uint32_t>(lane) < in_bin;
+          const uint32_t ck = s.cand[lane], ct = s.cand[32 + lane];  // past in_bin: unused
+          uint32_t rank = 0, gt = 0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t kj = __shfl_sync(0xffffffffu, ck, j);
+            const uint32_t tj = __shfl_sync(0xffffffffu, ct, j);
+            const bool valid = static_cast<uint32_t>(j) < in_bin;
+            rank += (valid && (kj > ck || (kj == ck && tj < ct))) ? 1u : 0u;
+            gt += (valid && kj > ck) ? 1u : 0u;
+          }
+          if (mine && rank == need - 1) {
+            s.sel[0] = ck;
+            s.sel[1] = need - gt;
+          }
+        }
+        __syncthreads();
+        T = s.sel[0];
+        need = s.sel[1];
+        break;
+      }
+      hb = shift - 1;
     }
-    __syncthreads();
-    prefix |= s.sel[2 * h] << shift;
-    mask |= 0xFFu << shift;
-    need -= s.sel[2 * h + 1];
-    ++pass;
   }
   // Ordered compaction: token t (first <= t < L) is kept when key_t > T, or key_t == T
   // and fewer than `need` equal keys precede it; its place among the kept tokens
-  // is (#keys > T before t) + min(#keys == T before t, need). One packed scan per
-  // round counts both (> T in the low half, == T in the high half).
-  const uint32_t T = prefix;  // the k-th largest key
+  // is (#keys > T before t) + min(#keys == T before t, need). One packed count per
+  // round (> T in the low half, == T in the high half): a warp scan, one barrier
+  // for the warp totals (double-buffered across rounds), each warp's own offset.
   uint32_t gt_base = 0, eq_base = 0;
-  for (int base = 0; base < L; base += 4 * nt) {
+  for (int base = 0, round = 0; base < L; base += 4 * nt, ++round) {
     const int t0 = base + 4 * tid;
     const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
     const uint32_t u[4] = {q.x, q.y, q.z, q.w};
@@ -389,10 +448,19 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
         eq_m |= static_cast<uint32_t>(u[i] == T) << i;
       }
     }
-    uint32_t tot;
-    const uint32_t pre =
-        block_exclusive_sum(static_cast<uint32_t>(__popc(gt_m)) | (static_cast<uint32_t>(__popc(eq_m)) << 16),
-                            s.warp, tot);
+    const uint32_t cnt = static_cast<uint32_t>(__popc(gt_m)) | (static_cast<uint32_t>(__popc(eq_m)) << 16);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    uint32_t* wb = s.warp + 32 * (round & 1);
+    if (lane == 31) wb[warp] = incl;
+    __syncthreads();
+    const uint32_t wt = lane < nw ? wb[lane] : 0u;
+    const uint32_t pre = __reduce_add_sync(0xffffffffu, lane < warp ? wt : 0u) + incl - cnt;
+    const uint32_t tot = __reduce_add_sync(0xffffffffu, wt);
     uint32_t gtb = gt_base + (pre & 0xFFFFu), eqb = eq_base + (pre >> 16);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -412,11 +480,12 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
                                                       float* __restrict__ scores,
                                                       int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[512], s_sel[4], s_rng[64];
+  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[64];
+  __shared__ __align__(16) uint32_t s_hist[768], s_cand[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
-  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng, s_cand);
   load_keys(partials, NP, L, b, scores, s, dist, cls ? 1 : 0);
   select_into_smem(L, k, s, cls);
   const int k1 = k + (cls ? 1 : 0);
@@ -477,12 +546,13 @@ __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_ga
     const uint4* __restrict__ y, int Cv, int S, float* __restrict__ scores,
     int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[33], s_hist[512], s_sel[4], s_rng[64];
+  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[64];
+  __shared__ __align__(16) uint32_t s_hist[768], s_cand[64];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x / S, j0 = blockIdx.x % S;
   const bool writer = j0 == 0;
-  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng);
+  const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng, s_cand);
   load_keys(partials, NP, L, b, writer ? scores : nullptr, s, dist, cls ? 1 : 0);
   select_into_smem(L, k, s, cls);
   const int k1 = k + (cls ? 1 : 0);

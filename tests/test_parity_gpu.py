@@ -98,8 +98,9 @@ def test_select_gather_equals_separate_steps(L, C, k):
 def test_select_gather_long_sequences(B, L, metric, cls):
     """The fused select+gather on long sequences (radix selection, several CTAs per
     sample when samples are few): the bits of the standalone selection
-    (rs_select_topk) and of the gather of its kept rows, on every keep_k edge, with
-    and without ties and a CLS token, for each distance."""
+    (rs_select_topk), the oracle's selection on the same fp32 scores, and the gather
+    of the kept rows, on every keep_k edge, with and without ties and a CLS token,
+    for each distance."""
     rs = _rs()
     C = 1024 if L <= 1569 else 128
     P = 6 if metric == "cosine" else 8
@@ -114,6 +115,10 @@ def test_select_gather_long_sequences(B, L, metric, cls):
             torch.cuda.synchronize()
             assert torch.equal(s1, s2), (B, L, k, "scores")
             assert torch.equal(k1, k2), (B, L, k, "kept_idx")
+            s_np = s2.cpu().numpy().astype(np.float64)
+            for b in range(B):
+                ref = oracle.select_topk(s_np[b], k, cls=cls)
+                assert k2[b].cpu().numpy().tolist() == ref.tolist(), (B, L, k, b, "vs oracle")
             ref = torch.stack([y[b][k1[b].long()] for b in range(B)]) if k1.shape[1] else yk
             assert torch.equal(yk, ref), (B, L, k, "y_kept")
     _device_ok()
