@@ -6,9 +6,12 @@
 // One CTA owns 128 queries of one (sample, head) and walks the keys in blocks
 // of 64 (online softmax); three CTAs share an SM (128 TMEM columns and ~65 KB of
 // shared memory each), so one CTA's softmax overlaps the others' loads and MMAs:
-//   warp 0      TMA producer: the Q tile once, then K and V tiles of each key
-//               block into a two-stage ring (3-D tensor maps over [B, L, 3C], so
-//               rows past a sample's L read as zero and never cross samples);
+//   warp 0      TMA producer: the Q tile once, then the K and V tiles of each key
+//               block into two-stage rings of their own (3-D tensor maps over
+//               [B, L, 3C], so rows past a sample's L read as zero and never cross
+//               samples). A K stage is free once its S MMA has finished and a V
+//               stage once its P V MMA has, so K_{j+2} is on its way while block j's
+//               softmax runs and neither ring waits on the other;
 //   warp 1      owns the CTA's TMEM columns and issues the MMAs:
 //               S_j = Q K_j^T (M = 128, N = 64, K = 64) into the TMEM score
 //               buffer, and O += P_j V_j (M = 128, N = 64, K = 64, V read MN-major)
@@ -62,8 +65,9 @@ __global__ void __launch_bounds__(kThreads, 3)
   uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + kPBytes);
   uint64_t* k_full = q_full + 1;
   uint64_t* v_full = k_full + kKvStages;
-  uint64_t* kv_empty = v_full + kKvStages;
-  uint64_t* s_full = kv_empty + kKvStages;
+  uint64_t* k_empty = v_full + kKvStages;
+  uint64_t* v_empty = k_empty + kKvStages;
+  uint64_t* s_full = v_empty + kKvStages;
   uint64_t* s_empty = s_full + 1;
   uint64_t* p_full = s_empty + 1;
   uint64_t* pv_full = p_full + 1;
@@ -85,7 +89,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     for (int s = 0; s < kKvStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, 4);
@@ -117,25 +122,33 @@ __global__ void __launch_bounds__(kThreads, 3)
       const int C = p.C;
       mbar_arrive_expect_tx(q_full, kBox);
       tma_load_3d(sQ, &tmQ, q_full, head * kHd, q0, b);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       const bool hook = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int s = j % kKvStages;
-        if (j >= kKvStages && !wait_bounded(&kv_empty[s], ((j / kKvStages) - 1) & 1, wc)) break;
-        // test hook: stop loading, so that the MMA warp's wait for this block runs out
-        if (hook && j == p.debug_skip_block) break;
-        mbar_arrive_expect_tx(&k_full[s], kKvBox);
-        tma_load_3d(sKs(s), &tmKV, &k_full[s], C + head * kHd, j * kKeys, b);
-        mbar_arrive_expect_tx(&v_full[s], kKvBox);
-        tma_load_3d(sVs(s), &tmKV, &v_full[s], 2 * C + head * kHd, j * kKeys, b);
-        issued = j + 1;
+      // K_j, then V_{j-1}: the S MMA of a block comes before its P V MMA
+      for (int j = 0; j <= nkb; ++j) {
+        if (j < nkb) {
+          const int s = j % kKvStages;
+          if (j >= kKvStages && !wait_bounded(&k_empty[s], ((j / kKvStages) - 1) & 1, wc)) break;
+          // test hook: stop loading, so that the MMA warp's wait for this block runs out
+          if (hook && j == p.debug_skip_block) break;
+          mbar_arrive_expect_tx(&k_full[s], kKvBox);
+          tma_load_3d(sKs(s), &tmKV, &k_full[s], C + head * kHd, j * kKeys, b);
+          k_issued = j + 1;
+        }
+        if (j >= 1) {
+          const int i = j - 1, s = i % kKvStages;
+          if (i >= kKvStages && !wait_bounded(&v_empty[s], ((i / kKvStages) - 1) & 1, wc)) break;
+          mbar_arrive_expect_tx(&v_full[s], kKvBox);
+          tma_load_3d(sVs(s), &tmKV, &v_full[s], 2 * C + head * kHd, i * kKeys, b);
+          v_issued = i + 1;
+        }
       }
       // every load issued has landed before the CTA may finish (after an abort too)
       wait_bounded(q_full, 0u, wc, false);
-      for (int j = issued > kKvStages ? issued - kKvStages : 0; j < issued; ++j) {
+      for (int j = k_issued > kKvStages ? k_issued - kKvStages : 0; j < k_issued; ++j)
         wait_bounded(&k_full[j % kKvStages], (j / kKvStages) & 1, wc, false);
+      for (int j = v_issued > kKvStages ? v_issued - kKvStages : 0; j < v_issued; ++j)
         wait_bounded(&v_full[j % kKvStages], (j / kKvStages) & 1, wc, false);
-      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -157,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 3)
                     sw128_mnmajor_desc(v_u32 + kk * 2048, kKvBox), kIdO,
                     (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(pv_full);
-        umma_commit(&kv_empty[st]);
+        umma_commit(&v_empty[st]);
         return true;
       };
       bool ok = wait_bounded(q_full, 0u, wc);
@@ -175,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 3)
           umma_bf16(tmem, sw128_kmajor_desc(q_u32) + kk * 2, sw128_kmajor_desc(k_u32) + kk * 2,
                     kIdS, kk > 0 ? 1u : 0u);
         umma_commit(s_full);
+        umma_commit(&k_empty[st]);
         if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
       if (ok) issue_pv(nkb - 1);
