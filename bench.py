@@ -67,7 +67,8 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- ncu traffic
 GEMM_SOURCES = ["free_vit_token_b200/csrc/rs_mlp.cu", "free_vit_token_b200/csrc/rs_ptx.cuh",
-                "free_vit_token_b200/csrc/rs_gelu_poly.h", "free_vit_token_b200/csrc/rs_internal.h"]
+                "free_vit_token_b200/csrc/rs_gelu.cuh", "free_vit_token_b200/csrc/rs_gelu_poly.h",
+                "free_vit_token_b200/csrc/rs_internal.h"]
 
 
 def gemm_source_hash() -> str:
