@@ -347,8 +347,7 @@ int rs_gather_rows(const void* y, int B, int L, int C, const int32_t* kept_idx, 
  *   Limits: M <= 65536 and H * C <= 4194304, beyond which it returns
  *   RS_ERR_SHAPE without launching (as for any other shape error).
  *   The first call on a device resolves the array's device address for that
- *   device (cudaGetSymbolAddress); make that first call before any stream
- *   capture begins.
+ *   device (cudaGetSymbolAddress) and keeps it.
  *   Every call on a device shares the one array and leaves its contents behind;
  *   each call writes every scratch byte it reads before reading it. The status
  *   slot starts at zero (the array is zero-initialised when the library loads)
