@@ -388,36 +388,53 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
         // ranks one of them against all (key descending, token ascending): the
         // need-th is the k-th ranked key overall, T its key, and the keys == T that
         // are kept are `need` minus the bin's keys above T; one barrier.
+        // (one shared atomic per warp round that holds any of them)
         for (int base = 0; base < L; base += 4 * nt) {
           const int t0 = base + 4 * tid;
           const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
           const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+          uint32_t bal[4], total = 0;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int t = t0 + i;
-            if (t >= first && t < L && ((u[i] - kmin) & mask) == prefix) {
-              const uint32_t slot = atomicAdd(&s.sel[6], 1u);
-              s.cand[slot] = u[i];
-              s.cand[32 + slot] = static_cast<uint32_t>(t);
+            bal[i] = __ballot_sync(0xffffffffu,
+                                   t >= first && t < L && ((u[i] - kmin) & mask) == prefix);
+            total += __popc(bal[i]);
+          }
+          if (total != 0u) {
+            uint32_t slot = 0;
+            if (lane == 0) slot = atomicAdd(&s.sel[6], total);
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+            const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if ((bal[i] >> lane) & 1u) {
+                const uint32_t at = slot + __popc(bal[i] & below);
+                s.cand[at] = u[i];
+                s.cand[32 + at] = static_cast<uint32_t>(t0 + i);
+              }
+              slot += __popc(bal[i]);
             }
           }
         }
         __syncthreads();
         if (warp == 0) {
-          // lane l holds candidate l; the others come by shuffle, one per step
+          // lane l holds candidate l as one 64-bit key, larger = ranked first (key
+          // descending, token ascending; tokens differ, so no two are equal); the others
+          // come by shuffle, one per step
           const bool mine = static_cast<uint32_t>(lane) < in_bin;
-          const uint32_t ck = s.cand[lane], ct = s.cand[32 + lane];  // past in_bin: unused
-          uint32_t rank = 0, gt = 0;
+          const uint64_t kk = mine ? (static_cast<uint64_t>(s.cand[lane]) << 32) |
+                                         static_cast<uint64_t>(~s.cand[32 + lane])
+                                   : 0ull;
+          uint32_t rank = 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const uint32_t kj = __shfl_sync(0xffffffffu, ck, j);
-            const uint32_t tj = __shfl_sync(0xffffffffu, ct, j);
-            const bool valid = static_cast<uint32_t>(j) < in_bin;
-            rank += (valid && (kj > ck || (kj == ck && tj < ct))) ? 1u : 0u;
-            gt += (valid && kj > ck) ? 1u : 0u;
-          }
-          if (mine && rank == need - 1) {
-            s.sel[0] = ck;
+          for (int j = 0; j < 32; ++j) rank += __shfl_sync(0xffffffffu, kk, j) > kk ? 1u : 0u;
+          // invalid lanes hold 0, below every candidate: they never count against one
+          const int at = __ffs(__ballot_sync(0xffffffffu, mine && rank == need - 1)) - 1;
+          const uint32_t tkey = static_cast<uint32_t>(__shfl_sync(0xffffffffu, kk, at) >> 32);
+          const uint32_t gt = __popc(__ballot_sync(0xffffffffu, mine && static_cast<uint32_t>(kk >> 32) > tkey));
+          if (lane == 0) {
+            s.sel[0] = tkey;
             s.sel[1] = need - gt;
           }
         }
