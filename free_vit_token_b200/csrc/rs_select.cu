@@ -130,7 +130,7 @@ struct SelSmem {
   uint32_t* hist;  // [3][256] radix histograms (pass p uses p % 3), zero on entry to a pass
   uint32_t* sel;   // [8]: [0] T and [1] need from the candidate ranking; [6] counts
                    // the keys listed in cand (zero on entry to the selection)
-  uint32_t* rng;   // [2 * 32] per warp: smallest and largest patch key it loaded
+  uint32_t* rng;   // [2]: the smallest and the largest ranked key of the sample
   uint32_t* cand;  // [2 * 32]: the final bin's keys [0, 32) and their tokens [32, 64)
 };
 
@@ -266,12 +266,25 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ partials, in
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if ((threadIdx.x & 31) == 0) {
-    s.rng[2 * (threadIdx.x >> 5)] = kmin;
-    s.rng[2 * (threadIdx.x >> 5) + 1] = kmax;
+    atomicMin(&s.rng[0], kmin);
+    atomicMax(&s.rng[1], kmax);
   }
-  for (int i = tid; i < 768; i += nt) s.hist[i] = 0;  // the radix histogram buffers
-  if (tid == 0) s.sel[6] = 0;
-  if (tid < 64) s.cand[tid] = 0u;
+  __syncthreads();
+}
+
+// The selection's shared state before its first use: range bounds, histograms,
+// candidate count and slots. Every thread calls it, before the kernel's
+// dependency wait (so it overlaps the previous kernel's tail); it ends with a
+// barrier.
+__device__ __forceinline__ void init_select_smem(uint32_t* s_hist, uint32_t* s_sel, uint32_t* s_rng,
+                                                 uint32_t* s_cand) {
+  for (int i = threadIdx.x; i < 768; i += blockDim.x) s_hist[i] = 0;
+  if (threadIdx.x < 64) s_cand[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) {
+    s_sel[6] = 0;
+    s_rng[0] = 0xFFFFFFFFu;
+    s_rng[1] = 0u;
+  }
   __syncthreads();
 }
 
@@ -305,16 +318,9 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
   // v = key - kmin in [0, kmax - kmin], which orders like the keys; its first digit
   // takes the 8 bits below the highest set bit of kmax - kmin, so it spreads the keys
   // over at least 128 bins however the range sits against powers of two (the fp32
-  // exponent field). Every warp reduces the per-warp ranges itself.
+  // exponent field).
   const int nw = nt >> 5;
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int i = lane; i < 2 * nw; i += 32) {
-    const uint32_t v = s.rng[i];
-    if (i & 1) hi = v > hi ? v : hi;
-    else lo = v < lo ? v : lo;
-  }
-  const uint32_t kmin = __reduce_min_sync(0xffffffffu, lo);
-  const uint32_t kmax = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t kmin = s.rng[0], kmax = s.rng[1];
   uint32_t T, need = static_cast<uint32_t>(k);  // keys == T kept, lowest index first
   if (kmin == kmax) {
     T = kmin;  // every ranked key is the same
@@ -497,9 +503,10 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
                                                       float* __restrict__ scores,
                                                       int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[64];
+  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[2];
   __shared__ __align__(16) uint32_t s_hist[768], s_cand[64];
   pdl_trigger();
+  init_select_smem(s_hist, s_sel, s_rng, s_cand);
   pdl_wait();
   const int b = blockIdx.x;
   const SelSmem s = carve(dyn, L, s_warp, s_hist, s_sel, s_rng, s_cand);
@@ -563,9 +570,10 @@ __global__ void __launch_bounds__(kSelGatherThreads, VPL >= 8 ? 1 : 2) select_ga
     const uint4* __restrict__ y, int Cv, int S, float* __restrict__ scores,
     int32_t* __restrict__ kept, uint4* __restrict__ y_kept) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[64];
+  __shared__ uint32_t s_warp[64], s_sel[8], s_rng[2];
   __shared__ __align__(16) uint32_t s_hist[768], s_cand[64];
   pdl_trigger();
+  init_select_smem(s_hist, s_sel, s_rng, s_cand);
   pdl_wait();
   const int b = blockIdx.x / S, j0 = blockIdx.x % S;
   const bool writer = j0 == 0;
