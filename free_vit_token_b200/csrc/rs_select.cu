@@ -659,9 +659,12 @@ cudaError_t launch_select_gather(const float* partials, int num_partials, const 
                                  int L, int C, int keep_k, int dist, bool cls, float* scores,
                                  int32_t* kept_idx, void* y_kept, int num_sms,
                                  cudaStream_t stream, bool pdl) {
-  // CTAs per sample: about one CTA per SM when B is small, one per sample otherwise
+  // CTAs per sample: about one CTA per SM when B is small, one per sample otherwise;
+  // where that leaves more than a tenth of the SMs without a CTA (B = 32 on 148 SMs:
+  // 128 CTAs), two per SM instead, which the copy's memory parallelism repays
   const int k1 = keep_k + (cls ? 1 : 0);
   int S = num_sms / B;
+  if (S >= 1 && 10 * B * S < 9 * num_sms && (C / 8 + 31) / 32 < 8) S = 2 * num_sms / B;
   if (S > k1) S = k1;
   if (S < 1) S = 1;
   const int Cv = C / 8;
