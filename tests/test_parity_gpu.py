@@ -124,6 +124,67 @@ def test_select_gather_long_sequences(B, L, metric, cls):
     _device_ok()
 
 
+def _crafted_keys(kind: str, n: int, g: torch.Generator) -> torch.Tensor:
+    """fp32 scores shaped to reach each branch of the radix selection."""
+    if kind == "all_equal":           # kmin == kmax: no pass at all
+        return torch.full((n,), 1.5)
+    if kind == "two_values":          # one pass, then bins of hundreds of equal keys
+        return torch.where(torch.rand(n, generator=g) < 0.5, torch.tensor(2.0), torch.tensor(3.0))
+    if kind == "one_outlier":         # the range is set by one key; the rest tie below it
+        v = torch.full((n,), 0.75)
+        v[n // 3] = 1e30
+        return v
+    if kind == "many_binades":        # scores from 2^-60 to 2^60, some exactly zero
+        v = torch.pow(2.0, torch.rand(n, generator=g) * 120 - 60)
+        v[torch.rand(n, generator=g) < 0.05] = 0.0
+        return v
+    if kind == "last_bits":           # keys that differ in their last few mantissa bits
+        base = torch.tensor(1.0).view(torch.int32).item()
+        return (base + torch.randint(0, 100, (n,), generator=g, dtype=torch.int32)).view(torch.float32)
+    if kind == "bin_of_32":           # 32 or 33 equal keys straddling the cut, the rest apart
+        v = torch.rand(n, generator=g) * 4.0 + 5.0
+        v[: n // 2] = torch.rand(n // 2, generator=g) * 0.5 + 0.5
+        v[n // 2: n // 2 + 33] = 2.0
+        return v
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("L", [257, 1569, 4100])
+@pytest.mark.parametrize("kind", ["all_equal", "two_values", "one_outlier", "many_binades",
+                                  "last_bits", "bin_of_32"])
+def test_select_crafted_key_distributions(L, kind):
+    """Key sets that drive the radix selection through each of its exits (no pass, the
+    full key reached, the final bin of at most 32 keys, bins of exactly 32 and 33): the
+    kept lists of the standalone and the fused selection, with and without CLS, at
+    every keep_k edge and around the 32-key bin, bit for bit against the oracle on the
+    same fp32 scores (L1 with one partial per row, so the score is the partial)."""
+    rs = _rs()
+    B, C = 3, 128
+    g = torch.Generator().manual_seed(L * 7 + len(kind))
+    parts = torch.stack([_crafted_keys(kind, L, g) for _ in range(B)]).reshape(B * L, 1)
+    pd = parts.to(dev)
+    y = torch.randn(B, L, C, generator=g).to(torch.bfloat16).to(dev)
+    for cls in (True, False):
+        nr = L - (1 if cls else 0)
+        half = L // 2 - (1 if cls else 0)
+        for k in sorted({0, 1, nr // 3, half - 1, half, half + 31, half + 32, half + 33, nr - 1, nr}):
+            if not 0 <= k <= nr:
+                continue
+            s1, k1 = rs.rs_select_topk(pd, B, L, k, distance="l1", cls=cls)
+            s2, k2, yk = rs.rs_select_gather(pd, y, k, distance="l1", cls=cls)
+            torch.cuda.synchronize()
+            assert torch.equal(s1.cpu().reshape(-1), parts.reshape(-1)), (kind, L, "scores")
+            assert torch.equal(k1, k2), (kind, L, k, cls)
+            s_np = s1.cpu().numpy().astype(np.float64)
+            for b in range(B):
+                ref = oracle.select_topk(s_np[b], k, cls=cls)
+                assert k1[b].cpu().numpy().tolist() == ref.tolist(), (kind, L, k, cls, b)
+            if k2.shape[1]:
+                ref_rows = torch.stack([y[b][k2[b].long()] for b in range(B)])
+                assert torch.equal(yk, ref_rows), (kind, L, k, cls, "rows")
+    _device_ok()
+
+
 # --------------------------------------------------------------------------- LN stats
 @pytest.mark.parametrize("C", [64, 192, 384, 768, 1024, 2048])
 def test_ln_stats(C):
