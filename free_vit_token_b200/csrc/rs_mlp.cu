@@ -12,11 +12,14 @@
 //         the L1 and cosine distances of §3.3: sum |h - x'|, or the triple
 //         (sum h x', sum h^2, sum x'^2) per column group
 //
-// One CTA per SM loops over 128 x BN output tiles. Warp roles:
+// One CTA per SM loops over 128 x BN output tiles (or a CTA pair over 256 x BN
+// tiles, tcgen05 cta_group::2, for long reductions). Warp roles:
 //   warp 0      TMA producer (A and B tiles, 64-wide K blocks, STAGES deep ring)
-//   warp 1      TMEM owner and UMMA issuer (tcgen05.mma, M=128, N=BN, K=16)
-//   warps 4-11  epilogue: TMEM -> registers -> LN fold / bias, GELU or
-//               residual/shift -> HBM (fc1 through per-warp TMA-store boxes)
+//   warp 1      TMEM owner and UMMA issuer (tcgen05.mma, M=128 or 256, N=BN, K=16)
+//   warps 2-3   idle (the epilogue's first warp sits on TMEM lane quadrant 0)
+//   warps 4-11  epilogue (4-19 for the folded-LN fc1 at C <= 512): TMEM ->
+//               registers -> LN fold / bias, GELU or residual/shift -> HBM through
+//               per-warp TMA-store boxes
 //   warps 12-15 (staged-LN fc1 only) LayerNorm staging of the A tile in place
 // The fp32 accumulator is double-buffered in TMEM (2 x BN columns) so the
 // epilogue of one tile overlaps the main loop of the next.
