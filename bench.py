@@ -474,6 +474,7 @@ def select_gather_times(blk, buf, flush_w, flush_r):
     rs, wl, dev, stream = blk.rs, blk.wl, blk.dev, blk.stream
     np_ = rs.rs_num_partials(wl.C)
     hot, cold = 0.0, 0.0
+    per_stage = []  # (hot ms, flushed ms) of each stage's launch
     cap_stream = torch.cuda.Stream(dev)
     for s, k in enumerate(wl.keep_k):
         L_s = wl.stage_L(s)
@@ -500,7 +501,8 @@ def select_gather_times(blk, buf, flush_w, flush_r):
             b.record(stream)
             torch.cuda.synchronize()
             reps.append(a.elapsed_time(b) / SG_REPS)
-        hot += statistics.median(reps)
+        hot_s = statistics.median(reps)
+        hot += hot_s
         del g
         gf, gfs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(gf, stream=cap_stream):
@@ -521,23 +523,27 @@ def select_gather_times(blk, buf, flush_w, flush_r):
                 torch.cuda.synchronize()
                 tt.append(a.elapsed_time(b))
             diffs.append(tt[1] - tt[0])
-        cold += max(statistics.median(diffs), 1e-6)
+        cold_s = max(statistics.median(diffs), 1e-6)
+        cold += cold_s
+        per_stage.append((hot_s, cold_s))
         del gf, gfs
     st = rs.rs_get_last_device_error()
     assert st == 0, rs.status_string(st)
-    return hot, cold
+    return hot, cold, per_stage
+
+
+def select_gather_stage_bytes(rs, wl, s: int) -> int:
+    """Algorithmic bytes of one stage's select+gather: the partials and the scores once,
+    kept_idx written, the kept rows read and written."""
+    np_ = rs.rs_num_partials(wl.C)
+    M, k = wl.tokens(s), wl.keep_k[s]
+    return (M * np_ * 4 + M * 4 + wl.B * (k + 1) * 4      # select: partials in, scores + idx out
+            + wl.B * (k + 1) * (4 + 2 * wl.C * 2))        # gather: idx in, rows in + out
 
 
 def select_gather_bytes(rs, wl) -> int:
-    """Algorithmic bytes of select+gather over every stage: the partials and the
-    scores once, kept_idx written, the kept rows read and written."""
-    np_ = rs.rs_num_partials(wl.C)
-    n = 0
-    for s, k in enumerate(wl.keep_k):
-        M = wl.tokens(s)
-        n += M * np_ * 4 + M * 4 + wl.B * (k + 1) * 4       # select: partials in, scores + idx out
-        n += wl.B * (k + 1) * (4 + 2 * wl.C * 2)           # gather: idx in, rows in + out
-    return n
+    """Algorithmic bytes of select+gather over every stage."""
+    return sum(select_gather_stage_bytes(rs, wl, s) for s in range(len(wl.keep_k)))
 
 
 def measure_block(blk, steps: int, warmup: int, l2_flush, flush_w, flush_r, world: int, peaks,
@@ -557,7 +563,7 @@ def measure_block(blk, steps: int, warmup: int, l2_flush, flush_w, flush_r, worl
         fc[n] = {"ms": kernel_ms[n], "tflops": tf, "frac": tf / peaks["bf16"],
                  "traffic": ncu_traffic(n, wl.name, wl.stages)}
     dominant = max(("fc1", "fc2"), key=lambda n: kernel_ms[n])
-    hot, cold = select_gather_times(blk, buf, flush_w, flush_r)
+    hot, cold, sg_stages = select_gather_times(blk, buf, flush_w, flush_r)
     sg_bytes = select_gather_bytes(rs, wl)
     block_flops = 2.0 * gemm_flops
     block_tf = block_flops / (ms_per_step / 1e3) / 1e12
@@ -579,7 +585,14 @@ def measure_block(blk, steps: int, warmup: int, l2_flush, flush_w, flush_r, worl
             "ms_single_launch_events": kernel_ms["select_gather"],
             "l2_hot": {"ms": hot, "GBps": gbs(hot), "frac_hbm": gbs(hot) / peaks["hbm"],
                        "timing": f"device time per launch, {SG_REPS} launches replayed from a "
-                                 "CUDA graph, inputs as fc2 left them (L2-resident)"}},
+                                 "CUDA graph, inputs as fc2 left them (L2-resident)"},
+            "per_stage": [
+                {"stage": i, "bytes": select_gather_stage_bytes(rs, wl, i),
+                 "ms": c, "frac_hbm": select_gather_stage_bytes(rs, wl, i) / (c / 1e3) / 1e9
+                 / peaks["hbm"],
+                 "l2_hot_ms": h, "l2_hot_frac_hbm": select_gather_stage_bytes(rs, wl, i)
+                 / (h / 1e3) / 1e9 / peaks["hbm"]}
+                for i, (h, c) in enumerate(sg_stages)] if wl.stages > 1 else None},
     }
 
 
