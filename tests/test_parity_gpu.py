@@ -401,6 +401,20 @@ def test_block_edges(B, L, C, H):
         parity.check_block(gpu, ref, k)
 
 
+@pytest.mark.parametrize("B,L,C,H", [(2, 65, 2048, 8192), (1, 130, 1024, 16384),
+                                     (3, 41, 2048, 2048)])
+def test_block_max_widths(B, L, C, H):
+    """The widest blocks the library accepts: C = 2048 (the widest LayerNorm row, eight
+    16-byte vectors per lane in the gather, CTA-pair GEMMs on both sides) and H = 16384
+    (256 k-blocks in fc2), against the oracle on every sample and keep_k edge."""
+    inp = random_block(B, L, C, H, seed=B + L + C + H, fg_rows=L // 3)
+    for k in (0, L // 2, L - 1):
+        gpu = _run_block(inp.x, inp.weights[0], k)
+        ref = parity.oracle_block(inp.x, inp.weights[0], k)
+        parity.check_block(gpu, ref, k)
+    _device_ok()
+
+
 def test_block_duplicate_rows_tie_rule():
     """Duplicated patch rows give identical scores on both sides; the lower index wins."""
     B, L, C, H = 2, 60, 192, 768
