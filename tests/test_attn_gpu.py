@@ -62,6 +62,21 @@ def test_attn_core_long():
     assert rs.rs_get_last_device_error() == 0
 
 
+@pytest.mark.parametrize("B,L,heads", [(1, 200, 32), (1, 4100, 1)])
+def test_attn_core_max_sizes(B, L, heads):
+    """32 heads (C = 2048, the widest accepted), and a sequence of 4100 tokens (65 key
+    blocks, a 4-row tail) against the fp64 core."""
+    rs = _rs()
+    qkv = random_qkv(B, L, heads, seed=L + heads, scale=1.5)
+    out = rs.rs_attn_core(qkv.to(dev), heads)
+    torch.cuda.synchronize()
+    got = parity.f64(out)
+    q64 = parity.f64(qkv)
+    for b in range(B):
+        parity.check_y(got[b], attn_oracle.attention_core(q64[b], heads), f"attn[{b}]")
+    assert rs.rs_get_last_device_error() == 0
+
+
 def test_attn_core_empty_batch():
     rs = _rs()
     qkv = torch.empty(0, 7, 3 * 128, dtype=torch.bfloat16, device=dev)
