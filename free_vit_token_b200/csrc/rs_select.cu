@@ -390,11 +390,11 @@ __device__ void select_into_smem(int L, int k, const SelSmem& s, bool cls) {
         break;
       }
       if (in_bin <= 32) {
-        // The bin's keys into s.cand in any order, one barrier; every lane of warp 0
-        // ranks one of them against all (key descending, token ascending): the
-        // need-th is the k-th ranked key overall, T its key, and the keys == T that
-        // are kept are `need` minus the bin's keys above T; one barrier.
-        // (one shared atomic per warp round that holds any of them)
+        // The bin's keys into s.cand in any order (one shared atomic per warp round
+        // that holds any of them), one barrier; every lane of warp 0 ranks one of them
+        // against all (key descending, token ascending): the need-th is the k-th
+        // ranked key overall, T its key, and the keys == T that are kept are `need`
+        // minus the bin's keys above T; one barrier.
         for (int base = 0; base < L; base += 4 * nt) {
           const int t0 = base + 4 * tid;
           const uint4 q = t0 < Lpad ? key4[t0 >> 2] : make_uint4(0, 0, 0, 0);
