@@ -16,7 +16,9 @@
 // tiles, tcgen05 cta_group::2, for long reductions). Warp roles:
 //   warp 0      TMA producer (A and B tiles, 64-wide K blocks, STAGES deep ring)
 //   warp 1      TMEM owner and UMMA issuer (tcgen05.mma, M=128 or 256, N=BN, K=16)
-//   warps 2-3   idle (the epilogue's first warp sits on TMEM lane quadrant 0)
+//   warp 2      each tile's column vectors (16-warp epilogue only; otherwise the
+//               producer loads them), warp 3 idle (the epilogue's first warp
+//               sits on TMEM lane quadrant 0)
 //   warps 4-11  epilogue (4-19 for the folded-LN fc1 at C <= 512): TMEM ->
 //               registers -> LN fold / bias, GELU or residual/shift -> HBM through
 //               per-warp TMA-store boxes
@@ -219,65 +221,84 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
 
+  // A tile's column vectors (the bias, or the LN fold's G and cb) go into the
+  // buffer of the accumulator it will use once the epilogue is done with that
+  // buffer's previous tile. The producer loads them at each tile's start, except
+  // with the 16-warp epilogue (short reductions): there the producer runs a whole
+  // tile ahead of that release, so warp 2 loads them and the operand stream never
+  // waits on the epilogue.
+  constexpr bool kVecWarp = EW == 16;
+  int vacc = 0;
+  uint32_t vphase = 0;
+  int vpend0 = -1, vpend1 = -1;
+  auto load_vectors = [&](int n_blk) -> bool {
+    if (!wait_bounded(&vempty[vacc], vphase ^ 1u, wc)) return false;
+    mbar_arrive_expect_tx(&vfull[vacc], kVecBytes);
+    uint8_t* vdst = sVec + vacc * kVecStride;
+    if constexpr (EPI == kEpiGeluFold) {
+      bulk_load(vdst, p.colG + n_blk * BN, BN * 4, &vfull[vacc]);
+      bulk_load(vdst + BN * 4, p.colC + n_blk * BN, BN * 4, &vfull[vacc]);
+    } else {
+      bulk_load(vdst, p.bias + n_blk * BN, BN * 2, &vfull[vacc]);
+    }
+    if (vacc == 0) vpend0 = static_cast<int>(vphase); else vpend1 = static_cast<int>(vphase);
+    if (++vacc == 2) { vacc = 0; vphase ^= 1u; }
+    return true;
+  };
+  // Every vector copy this thread issued must land before the CTA may exit.
+  auto finish_vectors = [&]() {
+    if (vpend0 >= 0) wait_bounded(&vfull[0], static_cast<uint32_t>(vpend0), wc, false);
+    if (vpend1 >= 0) wait_bounded(&vfull[1], static_cast<uint32_t>(vpend1), wc, false);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int vacc = 0;
-      uint32_t vphase = 0;
-      int pend[STAGES];
-      int vpend0 = -1, vpend1 = -1;
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) pend[s] = -1;
+      // stages with a copy in flight (bit s) and the phase it completes (bit s)
+      uint32_t pend_mask = 0, pend_phase = 0;
+      // both CTAs' loads of a pair complete on the leader's full barriers
+      const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(&full[0]), 0u) : 0u;
       for (int tile = unit0; tile < p.num_tiles; tile += units) {
         const int m_blk = tile / p.n_blocks, n_blk = tile % p.n_blocks;
-        // this tile's column vectors, into the buffer of the accumulator it will use
-        if (!wait_bounded(&vempty[vacc], vphase ^ 1u, wc)) break;
-        mbar_arrive_expect_tx(&vfull[vacc], kVecBytes);
-        uint8_t* vdst = sVec + vacc * kVecStride;
-        if constexpr (EPI == kEpiGeluFold) {
-          bulk_load(vdst, p.colG + n_blk * BN, BN * 4, &vfull[vacc]);
-          bulk_load(vdst + BN * 4, p.colC + n_blk * BN, BN * 4, &vfull[vacc]);
-        } else {
-          bulk_load(vdst, p.bias + n_blk * BN, BN * 2, &vfull[vacc]);
+        if constexpr (!kVecWarp) {
+          if (!load_vectors(n_blk)) break;
         }
-        if (vacc == 0) vpend0 = static_cast<int>(vphase); else vpend1 = static_cast<int>(vphase);
-        if (++vacc == 2) { vacc = 0; vphase ^= 1u; }
+        // test hook: leave one stage unfilled so the consumer's wait runs out
+        const int skip_kb = (blockIdx.x == 0 && tile == unit0) ? p.debug_skip_kb : -1;
+        const int a_row = m_blk * kTileM + static_cast<int>(rank) * kBM;
+        const int b_row = n_blk * BN + static_cast<int>(rank) * kBRows;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, wc)) { ok = false; break; }
-          // test hook: leave one stage unfilled so the consumer's wait runs out
-          const bool skip = kb == p.debug_skip_kb && blockIdx.x == 0 && tile == unit0;
-          if (!skip) {
+          if (kb != skip_kb) {
             if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
             if constexpr (PAIR) {
-              // both CTAs' loads complete on the leader's full barrier
-              const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0u);
-              tma_load_2d_pair(sA + stage * kAStageBytes, &tmA, fb, kb * kBK,
-                               m_blk * kTileM + static_cast<int>(rank) * kBM);
-              tma_load_2d_pair(sB + stage * kBStageBytes, &tmB, fb, kb * kBK,
-                               n_blk * BN + static_cast<int>(rank) * kBRows);
+              const uint32_t fb = full_leader + static_cast<uint32_t>(stage) * 8u;
+              tma_load_2d_pair(sA + stage * kAStageBytes, &tmA, fb, kb * kBK, a_row);
+              tma_load_2d_pair(sB + stage * kBStageBytes, &tmB, fb, kb * kBK, b_row);
             } else {
-              tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, m_blk * kBM);
-              tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, n_blk * BN);
+              tma_load_2d(sA + stage * kAStageBytes, &tmA, &full[stage], kb * kBK, a_row);
+              tma_load_2d(sB + stage * kBStageBytes, &tmB, &full[stage], kb * kBK, b_row);
             }
-            if (leader) {
-#pragma unroll
-              for (int s = 0; s < STAGES; ++s)
-                if (s == stage) pend[s] = static_cast<int>(phase);
-            }
+            const uint32_t bit = 1u << stage;
+            pend_mask |= bit;
+            pend_phase = (pend_phase & ~bit) | (phase << stage);
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
       }
-      // Every copy this thread issued must land before the CTA may exit.
+      // Every copy this thread issued must land before the CTA may exit (on a
+      // pair the non-leader's copies complete on the leader's barriers, which the
+      // leader waits for).
+      if (leader) {
 #pragma unroll
-      for (int s = 0; s < STAGES; ++s)
-        if (pend[s] >= 0) wait_bounded(&full[s], static_cast<uint32_t>(pend[s]), wc, false);
-      if (vpend0 >= 0) wait_bounded(&vfull[0], static_cast<uint32_t>(vpend0), wc, false);
-      if (vpend1 >= 0) wait_bounded(&vfull[1], static_cast<uint32_t>(vpend1), wc, false);
+        for (int s = 0; s < STAGES; ++s)
+          if (pend_mask & (1u << s)) wait_bounded(&full[s], (pend_phase >> s) & 1u, wc, false);
+      }
+      if constexpr (!kVecWarp) finish_vectors();
       if constexpr (PAIR) {
         // The leader's releases of every stage (multicast commits into this CTA's
         // empty barriers) have all arrived before the CTA may exit.
@@ -286,6 +307,14 @@ __global__ void __launch_bounds__(num_threads(LN_A, EW), 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+    }
+    __syncwarp();
+  } else if (kVecWarp && warp == 2) {
+    // ------------------------------------------------------------ column vectors
+    if (lane == 0) {
+      for (int tile = unit0; tile < p.num_tiles; tile += units)
+        if (!load_vectors(tile % p.n_blocks)) break;
+      finish_vectors();
     }
     __syncwarp();
   } else if (warp == 1) {
