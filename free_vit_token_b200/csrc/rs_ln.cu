@@ -109,25 +109,26 @@ __device__ __forceinline__ void ln_fold_body(const __nv_bfloat16* __restrict__ W
   const int nvec = C >> 3;
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
-  uint4 gv[VPL], bv[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int idx = lane + 32 * i;
-    gv[i] = idx < nvec ? __ldg(g4 + idx) : make_uint4(0, 0, 0, 0);
-    bv[i] = idx < nvec ? __ldg(b4 + idx) : make_uint4(0, 0, 0, 0);
-  }
   for (int j = gw0; j < H; j += nw) {
     const uint4* wr = reinterpret_cast<const uint4*>(W1 + static_cast<size_t>(j) * C);
     uint4* out = reinterpret_cast<uint4*>(Wg + static_cast<size_t>(j) * C);
+    // the row's weights first (HBM), then gamma and beta (L1/L2-resident, re-read per
+    // row rather than held in registers, so that the kernel keeps its occupancy)
+    uint4 wv[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int idx = lane + 32 * i;
+      wv[i] = idx < nvec ? __ldg(wr + idx) : make_uint4(0, 0, 0, 0);
+    }
     float gs = 0.f, cs = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int idx = lane + 32 * i;
       if (idx < nvec) {
-        const uint4 wv = __ldg(wr + idx);
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(&wv);
-        const uint32_t* g = reinterpret_cast<const uint32_t*>(&gv[i]);
-        const uint32_t* b = reinterpret_cast<const uint32_t*>(&bv[i]);
+        const uint4 gq = __ldg(g4 + idx), bq = __ldg(b4 + idx);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&wv[i]);
+        const uint32_t* g = reinterpret_cast<const uint32_t*>(&gq);
+        const uint32_t* b = reinterpret_cast<const uint32_t*>(&bq);
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
