@@ -401,6 +401,21 @@ def test_block_edges(B, L, C, H):
         parity.check_block(gpu, ref, k)
 
 
+def test_block_calls_of_changing_shapes():
+    """Calls of changing batch and length in a row, on the workspace the previous call
+    left, all match the oracle on every sample: 16 long samples (nine select+gather CTAs
+    per sample), a short batch, 400 short samples (more select+gather CTAs than fit on
+    the GPU at once), and the first shape again."""
+    cases = [(16, 300, 128, 256, 200), (3, 41, 128, 256, 20), (400, 9, 64, 128, 5),
+             (16, 300, 128, 256, 200)]
+    for i, (B, L, C, H, k) in enumerate(cases):
+        inp = random_block(B, L, C, H, seed=100 + i, fg_rows=L // 3)
+        gpu = _run_block(inp.x, inp.weights[0], k)
+        ref = parity.oracle_block(inp.x, inp.weights[0], k)
+        parity.check_block(gpu, ref, k)
+    _device_ok()
+
+
 @pytest.mark.parametrize("B,L,C,H", [(2, 65, 2048, 8192), (1, 130, 1024, 16384),
                                      (3, 41, 2048, 2048)])
 def test_block_max_widths(B, L, C, H):
